@@ -1,0 +1,125 @@
+"""Pins of the oracle's block quantiser, Smooth-QK calibration/application and the
+4-bit dot product (S) against library routines, invariants and closed forms."""
+import ml_dtypes
+import numpy as np
+import pytest
+
+from bit_flashattention_b200 import configs, gen
+
+
+def _dequant(codes, scales):
+    """Dequantise with ml_dtypes (library decode of E2M1 and E4M3)."""
+    lo = (codes & 0xF).astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    hi = (codes >> 4).astype(np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    v = np.stack([lo, hi], axis=-1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
+    s = scales.view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+    return v * np.repeat(s, 16, axis=-1)
+
+
+def test_block_amax_element_gets_top_code(orc):
+    # For a block whose scale is an E4M3 normal, amax/scale lies in 6*[1-2^-4, 1+2^-4],
+    # which E2M1 rounds to 6 (code 7): the largest element always uses the top code.
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((20000, 16)) * 10.0 ** rng.uniform(-1, 2, (20000, 1))).astype(np.float32)
+    codes, scales = orc.quant_blocks(x.ravel())
+    nib = np.stack([codes & 15, codes >> 4], -1).reshape(20000, 16)
+    top = np.abs(x).argmax(1)
+    assert np.all((nib[np.arange(20000), top] & 7) == 7)
+    assert np.all(scales >= 0x08)                    # normal E4M3 scales for these magnitudes
+
+
+def test_block_scale_equivariance(orc):
+    # Multiplying a block by 2^k (scale stays an E4M3 normal) leaves the codes unchanged
+    # and moves the scale's exponent by k: the scale really is amax/6 and codes use 1/scale.
+    rng = np.random.default_rng(5)
+    x = rng.uniform(-3, 3, (5000, 16)).astype(np.float32)
+    c0, s0 = orc.quant_blocks(x.ravel())
+    for k in (-3, 1, 4):
+        ck, sk = orc.quant_blocks((x * np.float32(2.0 ** k)).ravel())
+        assert np.array_equal(c0, ck)
+        assert np.array_equal(sk.astype(int) - s0.astype(int), np.full(s0.shape, 8 * k))
+
+
+def test_block_dequant_error_bound(orc):
+    # |x - dequant(x)| <= half the E2M1 gap at that magnitude times the scale (no saturation
+    # beyond the top code for amax, whose excess is bounded by the scale rounding).
+    rng = np.random.default_rng(6)
+    x = (rng.standard_normal(160000)).astype(np.float32)
+    codes, scales = orc.quant_blocks(x)
+    xd = _dequant(codes[None], scales[None])[0]
+    sig = np.repeat(scales.view(ml_dtypes.float8_e4m3fn).astype(np.float32), 16)
+    assert np.all(np.abs(x - xd) <= 1.0 * sig * 1.07 + 1e-30)
+    # relative Frobenius error of NVFP4 on Gaussian data is ~10%
+    assert np.linalg.norm(x - xd) / np.linalg.norm(x) < 0.15
+
+
+def test_quantize_rows_applies_group_channel_scale(orc):
+    # Power-of-two scales make x*s exact, so smoothing inside the quantiser must equal
+    # quantising the numpy product: pins the (kv group, channel) indexing of s.
+    B, H, Hkv, N, d = 2, 4, 2, 32, 64
+    rng = np.random.default_rng(7)
+    x = gen.f32_to_bf16_bits(rng.standard_normal((B, H, N, d)).astype(np.float32))
+    s = np.float32(2.0) ** rng.integers(-3, 4, (Hkv, d)).astype(np.float32)
+    c1, s1 = orc.quantize_rows(x, Hkv, s)
+    xs = gen.bf16_bits_to_f32(x) * np.repeat(s, H // Hkv, axis=0)[None, :, None, :]
+    c2, s2 = orc.quant_blocks(xs.ravel())
+    assert np.array_equal(c1.ravel(), c2) and np.array_equal(s1.ravel(), s2)
+
+
+def test_quantize_vt_is_blocks_along_tokens(orc):
+    B, Hkv, N, d = 1, 2, 64, 32
+    rng = np.random.default_rng(8)
+    v = gen.f32_to_bf16_bits(rng.standard_normal((B, Hkv, N, d)).astype(np.float32))
+    c1, s1 = orc.quantize_vt(v)
+    vt = np.ascontiguousarray(np.swapaxes(gen.bf16_bits_to_f32(v), 2, 3))
+    c2, s2 = orc.quant_blocks(vt.ravel())
+    assert np.array_equal(c1.ravel(), c2) and np.array_equal(s1.ravel(), s2)
+
+
+def test_calibrate_properties(orc):
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=8, Hkv=2, N=256)
+    q, k, _ = gen.inputs(w, calib=True)
+    s0, si0 = orc.calibrate(q, k, 0.0)
+    assert np.all(s0 == 1.0) and np.all(si0 == 1.0)            # alpha = 0 disables smoothing
+    s, si = orc.calibrate(q, k, 0.5)
+    assert np.array_equal(si, (np.float32(1.0) / s).astype(np.float32))
+    # balanced point: after smoothing, per-(group, channel) amax of Q*s and K/s agree
+    qf, kf = gen.bf16_bits_to_f32(q), gen.bf16_bits_to_f32(k)
+    grp = w.Hq // w.Hkv
+    aq = np.abs(qf).reshape(w.B, w.Hkv, grp, w.N, w.d).max(axis=(0, 2, 3))
+    ak = np.abs(kf).max(axis=(0, 2))
+    assert np.allclose(aq * s, ak / s, rtol=1e-6)
+    # scaling K by 4 (exact in bf16) scales s by 4^0.5 = 2 exactly
+    k4 = gen.f32_to_bf16_bits(kf * 4)
+    s4, _ = orc.calibrate(q, k4, 0.5)
+    assert np.array_equal(s4, s * 2)
+
+
+def test_s_dot_models_on_exact_cases(orc):
+    # With unit scales and small codes every partial sum is exact, so all three
+    # accumulation models must equal numpy's matmul of the dequantised operands.
+    rng = np.random.default_rng(9)
+    for d in (64, 128, 256):
+        qc = rng.integers(0, 256, (16, d // 2), dtype=np.uint8)
+        kc = rng.integers(0, 256, (24, d // 2), dtype=np.uint8)
+        qs = np.full((16, d // 16), 0x38, np.uint8)
+        ks = np.full((24, d // 16), 0x38, np.uint8)
+        ref = (_dequant(qc, qs).astype(np.float64) @ _dequant(kc, ks).astype(np.float64).T).astype(np.float32)
+        for model in (0, 1, 2):
+            assert np.array_equal(orc.qk_scores(qc, qs, kc, ks, model), ref)
+
+
+def test_s_dot_exact_model_is_rounded_exact_dot(orc):
+    # Scales within a 2^6 range keep the fp64 dot of dequantised values exact, so the
+    # "exact then one rounding" model must equal RN(numpy fp64 matmul).
+    rng = np.random.default_rng(10)
+    d = 128
+    qc = rng.integers(0, 256, (32, d // 2), dtype=np.uint8)
+    kc = rng.integers(0, 256, (40, d // 2), dtype=np.uint8)
+    qs = rng.integers(0x30, 0x50, (32, d // 16), dtype=np.uint8)
+    ks = rng.integers(0x30, 0x50, (40, d // 16), dtype=np.uint8)
+    ref = (_dequant(qc, qs).astype(np.float64) @ _dequant(kc, ks).astype(np.float64).T).astype(np.float32)
+    assert np.array_equal(orc.qk_scores(qc, qs, kc, ks, 2), ref)
+    for model in (0, 1):
+        got = orc.qk_scores(qc, qs, kc, ks, model).astype(np.float64)
+        assert np.all(np.abs(got - ref) <= 2 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64))
