@@ -105,7 +105,7 @@ def test_s_dot_models_on_exact_cases(orc):
         qs = np.full((16, d // 16), 0x38, np.uint8)
         ks = np.full((24, d // 16), 0x38, np.uint8)
         ref = (_dequant(qc, qs).astype(np.float64) @ _dequant(kc, ks).astype(np.float64).T).astype(np.float32)
-        for model in (0, 1, 2):
+        for model in (0, 1, 2, 3):
             assert np.array_equal(orc.qk_scores(qc, qs, kc, ks, model), ref)
 
 
@@ -123,3 +123,39 @@ def test_s_dot_exact_model_is_rounded_exact_dot(orc):
     for model in (0, 1):
         got = orc.qk_scores(qc, qs, kc, ks, model).astype(np.float64)
         assert np.all(np.abs(got - ref) <= 2 * np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64))
+
+
+def _rz_f32(num: int, den_log2: int) -> float:
+    """num * 2^-den_log2 rounded toward zero to fp32, with Python integers."""
+    a = abs(num)
+    n = a.bit_length()
+    if n > 24:
+        a = (a >> (n - 24)) << (n - 24)
+    return float(np.float32((-a if num < 0 else a) * 2.0 ** -den_log2))
+
+
+def test_s_dot_rz_model_against_integer_arithmetic(orc):
+    # Model 3 (per 64-chunk: acc = RZ(acc + exact chunk)) recomputed with Python big
+    # integers from the format definitions, on wide-range scales where rounding matters.
+    rng = np.random.default_rng(12)
+    E2 = [0, 1, 2, 3, 4, 6, 8, 12]
+    tw = lambda c: -E2[c & 7] if c & 8 else E2[c & 7]
+    sc = lambda b: (b & 7) if (b >> 3) == 0 else (8 + (b & 7)) << ((b >> 3) - 1)
+    for d in (64, 128, 256):
+        qc = rng.integers(0, 256, (8, d // 2), dtype=np.uint8)
+        kc = rng.integers(0, 256, (8, d // 2), dtype=np.uint8)
+        qs = rng.integers(1, 0x7F, (8, d // 16), dtype=np.uint8)
+        ks = rng.integers(1, 0x7F, (8, d // 16), dtype=np.uint8)
+        got = orc.qk_scores(qc, qs, kc, ks, 3)
+        for i in range(8):
+            for k in range(8):
+                qn = [(int(qc[i, e // 2]) >> (4 * (e & 1))) & 15 for e in range(d)]
+                kn = [(int(kc[k, e // 2]) >> (4 * (e & 1))) & 15 for e in range(d)]
+                acc = 0.0
+                for ch in range(d // 64):
+                    t = 0
+                    for b in range(4 * ch, 4 * ch + 4):
+                        isum = sum(tw(qn[16 * b + e]) * tw(kn[16 * b + e]) for e in range(16))
+                        t += isum * sc(int(qs[i, b])) * sc(int(ks[k, b]))
+                    acc = _rz_f32(int(round(acc * 2 ** 20)) + t, 20)
+                assert got[i, k] == np.float32(acc)
