@@ -1,0 +1,387 @@
+"""Benchmark of the HiFA4-style 4-bit attention forward on B200.
+
+One step = the whole hot path over one batch of the Qwen3-8B-shaped 4k causal workload
+(B=1, Hq=32, Hkv=8, N=4096, d=128): Smooth-QK + 4-bit quantisation of Q and K, 4-bit
+quantisation of V^T, and the fused 4-bit attention kernel, each launched through the C
+ABI (libhifa4.so).  Metric: TFLOPS = 4*B*Hq*N^2*d / 2 (causal) per step / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs the same per-GPU workload (weak scaling, no
+collective on the data path); value = flops of all ranks / max-over-ranks time.
+--impl reference times the CPU oracle (the reference arm of this build) on a bounded
+sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "qwen3-8b-4k"
+N_SETS = 6                      # rotated input sets: 6 x ~50 MB of bf16 inputs > 126 MB L2
+FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ---------------------------------------------------------------- host-side aggregation
+
+def aggregate(per_rank_ms, flops_per_rank_step, steps):
+    """Whole-job throughput from per-rank elapsed times: all ranks' flops / max time."""
+    world = len(per_rank_ms)
+    t = max(per_rank_ms)
+    return {"ms_total": t, "ms_per_step": t / steps,
+            "tflops": flops_per_rank_step * steps * world / (t * 1e-3) / 1e12}
+
+
+def reduce_max(value: float, dist=None, device=None) -> float:
+    """Max of a float over the ranks of the default process group (identity when single)."""
+    if dist is None or not dist.is_initialized():
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("hbm_gbs", FALLBACK_HBM_GBS), p.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples of one GPU while running."""
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hifa4_clocks_{os.getpid()}_{index}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons, n = [], [], set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                n += 1
+                for nm, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def make_inputs(w, device):
+    import numpy as np
+    import torch
+    from bit_flashattention_b200 import gen, hifa4
+    q, k, v = gen.inputs(w)
+    qc, kc, _ = gen.inputs(w, calib=True)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+    s, sinv = hifa4.hifa4_calibrate_smooth(dev(qc), dev(kc), w.alpha) if w.alpha is not None else (None, None)
+    base = (dev(q), dev(k), dev(v))
+    sets = [base] + [tuple(x.clone() for x in base) for _ in range(N_SETS - 1)]
+    host = tuple(torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).pin_memory()
+                 for a in (q, k, v))
+    return sets, host, s, sinv
+
+
+def run_gpu(args):
+    import torch
+    from bit_flashattention_b200 import configs, hifa4
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    w = configs.get(WORKLOAD)
+    flops = w.flops
+    sets, host, s, sinv = make_inputs(w, device)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    st = hifa4.new_status(device)
+    qq = [hifa4.QTensor(B, Hq, N, d, 0, device) for _ in range(2)]
+    kq = [hifa4.QTensor(B, Hkv, N, d, 0, device) for _ in range(2)]
+    vq = [hifa4.QTensor(B, Hkv, N, d, 1, device) for _ in range(2)]
+    o = torch.empty(B, Hq, N, d, dtype=torch.bfloat16, device=device)
+    m = torch.empty(B, Hq, N, dtype=torch.float16, device=device)
+    l = torch.empty(B, Hq, N, dtype=torch.float16, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        qt, kt, vt = sets[i % N_SETS]
+        j = i & 1
+        if ev is not None:
+            ev[0].record(stream)
+        hifa4.hifa4_quantize_qk(qt, kt, s, sinv, status=st, out=(qq[j], kq[j]))
+        if ev is not None:
+            ev[1].record(stream)
+        hifa4.hifa4_quantize_v(vt, status=st, out=vq[j])
+        if ev is not None:
+            ev[2].record(stream)
+        hifa4.hifa4_attn_fwd_quantized(qq[j], kq[j], vq[j], causal=w.causal, kv_tile=w.bc, status=st, o=o, m=m, l=l)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    code = hifa4.hifa4_read_status(st)
+    if code != hifa4.OK:
+        raise RuntimeError(f"warm-up reported {hifa4.status_string(code)}")
+
+    # timed region: K steps, barrier + synchronize on both sides, per-kernel events inside
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        step(i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed = t_begin.elapsed_time(t_end)
+    code = hifa4.hifa4_read_status(st)
+    if code != hifa4.OK:
+        raise RuntimeError(f"timed steps reported {hifa4.status_string(code)}")
+    k_qk = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    k_v = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    k_attn = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+
+    # e2e through the public API with host buffers: H2D of Q, K, V from pinned memory,
+    # the hot path, D2H of O, m, l -- every step
+    e2e_steps = max(3, min(args.steps, 20))
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    mh = torch.empty(m.shape, dtype=m.dtype, pin_memory=True)
+    lh = torch.empty(l.shape, dtype=l.dtype, pin_memory=True)
+    qd, kd, vd = sets[0]
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        qd.copy_(host[0], non_blocking=True)
+        kd.copy_(host[1], non_blocking=True)
+        vd.copy_(host[2], non_blocking=True)
+        step(0)
+        oh.copy_(o, non_blocking=True)
+        mh.copy_(m, non_blocking=True)
+        lh.copy_(l, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    elapsed = reduce_max(elapsed, dist, device)
+    e2e_ms = reduce_max(e2e_ms, dist, device)
+    k_attn = reduce_max(k_attn, dist, device)
+    k_qk = reduce_max(k_qk, dist, device)
+    k_v = reduce_max(k_v, dist, device)
+    agg = aggregate([elapsed] * world, flops, args.steps)
+    e2e = aggregate([e2e_ms] * world, flops, e2e_steps)
+    h2d = sum(x.numel() * x.element_size() for x in host)
+    d2h = sum(x.numel() * x.element_size() for x in (oh, mh, lh))
+
+    hbm, bf16, src = peaks()
+    fp4_peak = bf16 * FP4_OVER_BF16
+    achieved = flops / (k_attn * 1e-3) / 1e12
+    qk_bytes = (B * (Hq + Hkv) * N * d) * (2 + 0.5 + 1 / 16)
+    out = {
+        "metric": "4-bit attn fwd TFLOPS (4*B*Hq*N^2*d, causal/2) and % of B200 dense FP4 peak",
+        "value": round(agg["tflops"], 3),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(agg["ms_per_step"], 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp4_e2m1 (ue4m3 block scales), fp32 accumulate, fp16 softmax state",
+        "data": "synthetic (seeded Qwen3-8B-shaped post-RoPE Q/K/V, K outlier channels + bias)",
+        "config": {"workload": WORKLOAD, "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
+                   "kv_tile": w.bc, "smooth_qk_alpha": w.alpha,
+                   "l2": f"inputs rotated over {N_SETS} buffer sets (> 126 MB L2)", "parallelism": f"replicas x{world}"},
+        "pct_fp4_peak": round(100 * agg["tflops"] / world / fp4_peak, 2),
+        "pct_fp4_peak_datasheet_9pf": round(100 * agg["tflops"] / world / 9000.0, 2),
+        "tokens_per_s": round(B * N * world / (agg["ms_per_step"] * 1e-3), 1),
+        "kernels_us": {"quantize_qk": round(k_qk * 1e3, 2), "quantize_v": round(k_v * 1e3, 2),
+                       "attn_fwd": round(k_attn * 1e3, 2)},
+        "attn_kernel_tflops": round(achieved, 2),
+        "quantize_qk_gbs": round(qk_bytes / (k_qk * 1e-3) / 1e9, 1),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "peak_source": f"{src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)"},
+        "e2e": {"value": round(e2e["tflops"], 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+# ---------------------------------------------------------------- CPU oracle arm
+
+def _oracle_setup(w):
+    import oracle
+    from bit_flashattention_b200 import gen
+    q, k, v = gen.inputs(w)
+    s = sinv = None
+    if w.alpha is not None:
+        qc, kc, _ = gen.inputs(w, calib=True)
+        s, sinv = oracle.calibrate(qc, kc, w.alpha)
+    return q, k, v, s, sinv
+
+
+def _oracle_step(w, data, qtile, head):
+    """Oracle forward of one 128-row query tile of one (batch, head): Smooth-QK + 4-bit
+    quantisation of that head's Q and of its kv head's K and V^T, then the tile's rows."""
+    import numpy as np
+    import oracle
+    q, k, v, s, sinv = data
+    b, h = divmod(head, w.Hq)
+    g = h // (w.Hq // w.Hkv)
+    sl = lambda a, hh: np.ascontiguousarray(a[b:b + 1, hh:hh + 1])
+    sg = None if s is None else s[g:g + 1]
+    sig = None if sinv is None else sinv[g:g + 1]
+    qz = oracle.quantize_all(sl(q, h), sl(k, g), sl(v, g), sg, sig)
+    rows = np.arange(qtile * 128, qtile * 128 + 128, dtype=np.int64)
+    oracle.attn_fwd(qz, w.causal, w.bc, rows)
+    keys = sum((qtile * 128 + i + 1) if w.causal else w.N for i in range(128))
+    return 4.0 * w.d * keys
+
+
+def cpu_baseline(w, budget_s=15.0):
+    import oracle
+    data = _oracle_setup(w)
+    done_flops, t = 0.0, 0.0
+    n = 0
+    nqt = w.N // 128
+    while t < budget_s and n < 256:
+        t0 = time.perf_counter()
+        done_flops += _oracle_step(w, data, (n * 7 + 3) % nqt, (n * 5) % (w.B * w.Hq))
+        t += time.perf_counter() - t0
+        n += 1
+    return {"value": round(done_flops / t / 1e12, 6), "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} steps of {WORKLOAD}, each one 128-row query tile of one head (seeded spread over heads "
+                      f"and tile positions) including the oracle's quantisation of that head's Q, K and V^T; "
+                      f"{t:.1f} s of CPU time"}
+
+
+def run_reference(args):
+    import oracle
+    from bit_flashattention_b200 import configs
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    w = configs.get(WORKLOAD)
+    data = _oracle_setup(w)
+    nqt = w.N // 128
+    for i in range(min(args.warmup, 3)):
+        _oracle_step(w, data, (i * 7 + 3) % nqt, 0)
+    flops, t = 0.0, 0.0
+    steps = min(args.steps, 200)
+    for i in range(steps):
+        t0 = time.perf_counter()
+        flops += _oracle_step(w, data, (i * 7 + 3) % nqt, (i * 5) % (w.B * w.Hq))
+        t += time.perf_counter() - t0
+    value = flops / t / 1e12
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    out = {
+        "impl": "reference",
+        "metric": "4-bit attn fwd TFLOPS (4*B*Hq*N^2*d, causal/2) and % of B200 dense FP4 peak",
+        "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t / steps, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp4_e2m1 (ue4m3 block scales), exact sums, fp16 softmax state",
+        "data": "synthetic (seeded Qwen3-8B-shaped post-RoPE Q/K/V)",
+        "config": {"workload": WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+                   "kv_tile": w.bc, "parallelism": "cpu oracle"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{steps} steps, each one 128-row query tile of one head including the oracle's "
+                                   "quantisation of that head's Q, K and V^T"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="hifa4", choices=["hifa4", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

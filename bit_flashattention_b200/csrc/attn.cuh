@@ -1,0 +1,633 @@
+// Fused 4-bit attention forward for sm_100a ("HiFA4: Training-Free 4-bit FlashAttention on
+// Ascend HIF4 NPUs for LLM Inference", abstract): QK^T and PV both run as block-scaled
+// FP4 tensor-core MMAs (tcgen05 kind::mxf4nvf4, accumulators in TMEM), the online-softmax
+// running max m and normaliser l are kept in FP16, P is quantised to the 4-bit P_hat in
+// registers, and -- P-Reordering -- the normaliser is summed from that same P_hat by the
+// tensor core: an extra MMA of P_hat against a block of ones (N = 16) runs next to the
+// PV MMA, so no row sum of P is computed on the ALUs.
+//
+// One CTA works on one (batch, query head, 128-row query tile); kv tiles of BC keys are
+// visited in ascending order.  Warp roles:
+//   warp 0      TMA producer: Q tile once, then K and V^T tiles (+ their scale atoms)
+//               into KS / VS-deep shared-memory rings.
+//   warp 1      allocates TMEM; lane 0 issues tcgen05.cp (scales -> TMEM) and MMAs:
+//               S_j = Q K_j^T into a double-buffered S, then O += P_hat_j V_j and
+//               R = P_hat_j * ones.
+//   warps 2..5  softmax: thread = one query row (TMEM lane).  Per tile: load S row, mask,
+//               m_new = max(m, fp16(rowmax(S) * c)), P = E(fma(S, c, -m_new)) quantised to
+//               P_hat (codes -> shared memory in the MMA's swizzled layout, scales -> a
+//               scale atom), then after PV_{j-1} completed: l = fp16(fma(alpha_{j-1}, l,
+//               R)) and O *= alpha_j where m changed.  Epilogue O / l -> bf16.
+// Every wait is bounded (wall-clock limit, shared abort flag); on a timeout the kernel
+// sets the status word, drains its own copies and MMAs and frees TMEM before exiting.
+#pragma once
+#include <cuda.h>
+#include "method.cuh"
+
+namespace hifa4 {
+
+__host__ __device__ constexpr uint32_t layout_code(int rowbytes) {
+  return rowbytes == 32 ? 6u : rowbytes == 64 ? 4u : 2u;   // UMMA SWIZZLE_32B / 64B / 128B
+}
+__host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+template <int D_, int BC_>
+struct AttnCfg {
+  static constexpr int D = D_, BC = BC_, BR = 128;
+  static constexpr int KQ = D / 64;             // 64-wide K chunks of QK^T
+  static constexpr int KP = BC / 64;            // 64-wide K chunks of PV
+  static constexpr int NAV = (D + 127) / 128;   // 128-channel scale atoms of V^T
+  static constexpr int QROW = D / 2, PROW = BC / 2;
+  static constexpr int KS = 3, VS = 3;
+  static constexpr uint32_t LQ = layout_code(QROW), LP = layout_code(PROW);
+  static constexpr uint32_t SZ_Q = BR * QROW, SZ_K = BC * QROW, SZ_V = D * PROW, SZ_P = BR * PROW;
+  static constexpr uint32_t SZ_ONES = 16 * PROW;
+  static constexpr uint32_t SZ_QSF = KQ * 512, SZ_KSF = KQ * 512, SZ_VSF = KP * NAV * 512, SZ_PSF = KP * 512;
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + align_up(SZ_Q, 1024);
+  static constexpr uint32_t OFF_V = OFF_K + KS * align_up(SZ_K, 1024);
+  static constexpr uint32_t OFF_P = OFF_V + VS * align_up(SZ_V, 1024);
+  static constexpr uint32_t OFF_ONES = OFF_P + 2 * align_up(SZ_P, 1024);
+  static constexpr uint32_t OFF_QSF = OFF_ONES + align_up(SZ_ONES, 1024);
+  static constexpr uint32_t OFF_KSF = OFF_QSF + SZ_QSF;
+  static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
+  static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
+  static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
+  static constexpr uint32_t OFF_BAR = OFF_1SF + 512;
+  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
+  // s_empty[2], p_full[2], o_bar, drain
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 6 + 2;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
+  static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-B alignment
+  // TMEM columns
+  static constexpr uint32_t T_S = 0, T_O = 2 * BC, T_R = T_O + D, T_SFQ = T_R + 16;
+  static constexpr uint32_t T_SFK = T_SFQ + 4 * KQ, T_SFP = T_SFK + 8 * KQ, T_SFV = T_SFP + 8 * KP;
+  static constexpr uint32_t T_SF1 = T_SFV + 8 * KP * NAV, T_END = T_SF1 + 4;
+  static constexpr uint32_t TMEM_COLS = T_END <= 256 ? 256 : 512;
+  static_assert(T_END <= 512, "TMEM budget exceeded");
+  static_assert(D == 64 || D == 128 || D == 256, "head dim");
+  static_assert(BC == 64 || BC == 128, "kv tile");
+  static constexpr int NTHREADS = 192;
+};
+
+struct AttnParams {
+  const uint8_t* qsf;       // Q scale atoms  [B, Hq, N/128, D/64, 512]
+  const uint8_t* ksf;       // K scale atoms  [B, Hkv, N/128, D/64, 512]
+  const uint8_t* vsf;       // V^T scale atoms [B, Hkv, N/64, ceil(D/128), 512]
+  __nv_bfloat16* o;         // [B, Hq, N, D]
+  __half* m_out;            // [B, Hq, N] or nullptr
+  __half* l_out;            // [B, Hq, N] or nullptr
+  int* status;
+  int B, Hq, Hkv, N, causal;
+  float c;                  // RN(log2(e) / sqrt(D))
+  unsigned long long wait_ns;
+  int inject;               // 1: the producer never delivers kv tile 1 (timeout test)
+};
+
+// Keep the register results of tcgen05.ld from being read before tcgen05.wait::ld.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Bounded wait that also returns early when another role aborted; warp-uniform result.
+__device__ __forceinline__ bool wait_all(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                         uint64_t ns) {
+  bool ok = mbar_wait(bar, parity, abort, status, ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait used while draining: ignores the abort flag.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t ns) {
+  int never = 0;
+  return mbar_wait(bar, parity, &never, status, ns);
+}
+
+template <int D, int BC>
+__global__ void __launch_bounds__(192, 1)
+    k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+  using C = AttnCfg<D, BC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sOnes = smem + C::OFF_ONES;
+  uint8_t* sQsf = smem + C::OFF_QSF;
+  uint8_t* s1sf = smem + C::OFF_1SF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::KS;
+  uint64_t* v_full = k_empty + C::KS;
+  uint64_t* v_empty = v_full + C::VS;
+  uint64_t* s_full = v_empty + C::VS;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* o_bar = p_full + 2;
+  uint64_t* drain_bar = o_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  auto sK = [&](int s) { return smem + C::OFF_K + s * align_up(C::SZ_K, 1024); };
+  auto sV = [&](int s) { return smem + C::OFF_V + s * align_up(C::SZ_V, 1024); };
+  auto sP = [&](int s) { return smem + C::OFF_P + s * align_up(C::SZ_P, 1024); };
+  auto sKsf = [&](int s) { return smem + C::OFF_KSF + s * C::SZ_KSF; };
+  auto sVsf = [&](int s) { return smem + C::OFF_VSF + s * C::SZ_VSF; };
+  auto sPsf = [&](int s) { return smem + C::OFF_PSF + s * C::SZ_PSF; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = p.B * p.Hq;
+  const int nqt = p.N / 128;
+  const int qtile = p.causal ? nqt - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x / BH);
+  const int bh = blockIdx.x % BH;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int nt = p.causal ? ((qtile + 1) * 128) / BC : p.N / BC;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NBAR; ++i) {
+      const bool four = (&bars[i] == &s_empty[0] || &bars[i] == &s_empty[1] || &bars[i] == &p_full[0] ||
+                         &bars[i] == &p_full[1]);
+      mbar_init(&bars[i], four ? 4 : 1);   // s_empty / p_full: one arrival per softmax warp
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp >= 2) {
+    // the ones operand (E2M1 1.0 = 0b0010 in both nibbles) and its scales (UE4M3 1.0)
+    for (int i = threadIdx.x - 64; i < (int)C::SZ_ONES / 4; i += 128) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
+    for (int i = threadIdx.x - 64; i < 128; i += 128) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(q_full, C::SZ_Q + C::SZ_QSF);
+      tma_load_2d(sQ, &tmQ, 0, bh * p.N + qtile * 128, q_full);
+      bulk_load(sQsf, p.qsf + ((long long)bh * nqt + qtile) * C::SZ_QSF, C::SZ_QSF, q_full);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        if (p.inject == 1 && j == 1) break;
+        const int ks = j % C::KS, vs = j % C::VS;
+        if (j >= C::KS && !mbar_wait(&k_empty[ks], ((j / C::KS) - 1) & 1, abort, p.status, p.wait_ns)) break;
+        mbar_arrive_expect_tx(&k_full[ks], C::SZ_K + C::SZ_KSF);
+        tma_load_2d(sK(ks), &tmK, 0, kvh * p.N + j * BC, &k_full[ks]);
+        const int katom = (j * BC) / 128;
+        bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * C::SZ_KSF, C::SZ_KSF, &k_full[ks]);
+        if (j >= C::VS && !mbar_wait(&v_empty[vs], ((j / C::VS) - 1) & 1, abort, p.status, p.wait_ns)) {
+          issued = 2 * j + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[vs], C::SZ_V + C::SZ_VSF);
+        tma_load_2d(sV(vs), &tmV, j * C::PROW, kvh * D, &v_full[vs]);
+        bulk_load(sVsf(vs), p.vsf + ((long long)kvh * (p.N / 64) + j * C::KP) * (C::NAV * 512), C::SZ_VSF,
+                  &v_full[vs]);
+        issued = 2 * j + 2;
+      }
+      // drain: every load this warp issued must have landed before the CTA exits
+      drain_wait(q_full, 0, p.status, p.wait_ns);
+      const int nk = (issued + 1) / 2, nv = issued / 2;
+      for (int s = 0; s < C::KS && s < nk; ++s) {
+        const int last = s + ((nk - 1 - s) / C::KS) * C::KS;
+        drain_wait(&k_full[s], (last / C::KS) & 1, p.status, p.wait_ns);
+      }
+      for (int s = 0; s < C::VS && s < nv; ++s) {
+        const int last = s + ((nv - 1 - s) / C::VS) * C::VS;
+        drain_wait(&v_full[s], (last / C::VS) & 1, p.status, p.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t ID_QK = idesc_nvf4(128, BC), ID_PV = idesc_nvf4(128, D), ID_R = idesc_nvf4(128, 16);
+    const uint32_t aQ = smem_u32(sQ), aOnes = smem_u32(sOnes);
+    auto issue_pv = [&](int t) -> bool {
+      const int vs = t % C::VS, pb = t & 1;
+      bool ok = wait_all(&v_full[vs], (t / C::VS) & 1, abort, p.status, p.wait_ns);
+      ok = ok && wait_all(&p_full[pb], (t >> 1) & 1, abort, p.status, p.wait_ns);
+      if (!ok) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sfv = tbase + C::T_SFV + pb * 4 * C::KP * C::NAV;
+        const uint32_t sfp = tbase + C::T_SFP + pb * 4 * C::KP;
+#pragma unroll
+        for (int i = 0; i < C::KP * C::NAV; ++i) tmem_cp_sf_atom(sfv + 4 * i, sVsf(vs) + 512 * i);
+#pragma unroll
+        for (int kc = 0; kc < C::KP; ++kc) tmem_cp_sf_atom(sfp + 4 * kc, sPsf(pb) + 512 * kc);
+        const uint32_t aP = smem_u32(sP(pb)), aV = smem_u32(sV(vs));
+#pragma unroll
+        for (int kc = 0; kc < C::KP; ++kc)
+          mma_nvf4(tbase + C::T_O, smem_desc(aP + 32 * kc, 0, 8 * C::PROW, C::LP),
+                   smem_desc(aV + 32 * kc, 0, 8 * C::PROW, C::LP), ID_PV, sfp + 4 * kc, sfv + 4 * C::NAV * kc,
+                   (t > 0 || kc > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kc = 0; kc < C::KP; ++kc)
+          mma_nvf4(tbase + C::T_R, smem_desc(aP + 32 * kc, 0, 8 * C::PROW, C::LP),
+                   smem_desc(aOnes + 32 * kc, 0, 8 * C::PROW, C::LP), ID_R, sfp + 4 * kc, tbase + C::T_SF1,
+                   kc > 0 ? 1u : 0u);
+        tc_commit(o_bar);
+        tc_commit(&v_empty[vs]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = wait_all(q_full, 0, abort, p.status, p.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      if (lane == 0) {
+#pragma unroll
+        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(tbase + C::T_SFQ + 4 * kc, sQsf + 512 * kc);
+        tmem_cp_sf_atom(tbase + C::T_SF1, s1sf);
+      }
+      __syncwarp();
+    }
+    for (int j = 0; ok && j < nt; ++j) {
+      const int ks = j % C::KS, sb = j & 1;
+      ok = wait_all(&k_full[ks], (j / C::KS) & 1, abort, p.status, p.wait_ns);
+      if (ok && j >= 2) ok = wait_all(&s_empty[sb], ((j >> 1) - 1) & 1, abort, p.status, p.wait_ns);
+      if (!ok) break;
+      if (BC == 64 && (j & 1)) {
+        // keys 64..127 of the 128-row scale atom: move record words 2,3 into words 0,1
+#pragma unroll
+        for (int kc = 0; kc < C::KQ; ++kc) {
+          uint4* rec = reinterpret_cast<uint4*>(sKsf(ks) + 512 * kc) + lane;
+          uint4 w = *rec;
+          *rec = make_uint4(w.z, w.w, w.z, w.w);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t sfk = tbase + C::T_SFK + sb * 4 * C::KQ;
+#pragma unroll
+        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(sfk + 4 * kc, sKsf(ks) + 512 * kc);
+        const uint32_t aK = smem_u32(sK(ks));
+#pragma unroll
+        for (int kc = 0; kc < C::KQ; ++kc)
+          mma_nvf4(tbase + C::T_S + sb * BC, smem_desc(aQ + 32 * kc, 0, 8 * C::QROW, C::LQ),
+                   smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc, sfk + 4 * kc,
+                   kc > 0 ? 1u : 0u);
+        tc_commit(&s_full[sb]);
+        tc_commit(&k_empty[ks]);
+      }
+      __syncwarp();
+      if (j >= 1) ok = issue_pv(j - 1);
+    }
+    if (ok) ok = issue_pv(nt - 1);
+    // drain: every MMA / copy this warp issued has completed before TMEM is freed
+    if (lane == 0) {
+      tc_commit(drain_bar);
+      drain_wait(drain_bar, 0, p.status, p.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
+    const int qrow = qtile * 128 + row;
+    const float c = p.c;
+    float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int sb = j & 1;
+      ok = wait_all(&s_full[sb], (j >> 1) & 1, abort, p.status, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      float s[BC];
+      {
+        uint32_t r[BC];
+#pragma unroll
+        for (int c0 = 0; c0 < BC; c0 += 32)
+          tmem_ld32(tbase + lrow + C::T_S + sb * BC + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+        tmem_wait_ld();
+        reg_fence(r);
+#pragma unroll
+        for (int i = 0; i < BC; ++i) s[i] = __uint_as_float(r[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[sb]);
+      if (p.causal && (j + 1) * BC - 1 > qtile * 128) {
+#pragma unroll
+        for (int i = 0; i < BC; ++i)
+          if (j * BC + i > qrow) s[i] = -INFINITY;
+      }
+      float bmax[BC / 16];
+#pragma unroll
+      for (int bl = 0; bl < BC / 16; ++bl) {
+        float m = s[bl * 16];
+#pragma unroll
+        for (int e = 1; e < 15; e += 2) m = fmax3(m, s[bl * 16 + e], s[bl * 16 + e + 1]);
+        bmax[bl] = fmaxf(m, s[bl * 16 + 15]);
+      }
+      float rmax = bmax[0];
+#pragma unroll
+      for (int bl = 1; bl < BC / 16; ++bl) rmax = fmaxf(rmax, bmax[bl]);
+      float mnew = m_run;
+      if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
+      const float alpha = (m_run == -INFINITY) ? 0.0f : exp2_own(__fsub_rn(m_run, mnew));
+      const float negm = -mnew;
+      uint32_t words[BC / 8];
+      uint32_t sfw[C::KP];
+#pragma unroll
+      for (int kc = 0; kc < C::KP; ++kc) sfw[kc] = 0;
+#pragma unroll
+      for (int bl = 0; bl < BC / 16; ++bl) {
+        float R;
+        const uint32_t sc = block_scale(exp2_own(__fmaf_rn(bmax[bl], c, negm)), R);
+        sfw[bl / 4] |= sc << (8 * (bl % 4));
+        float x0[8], x1[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x0[e] = exp2_own(__fmaf_rn(s[bl * 16 + e], c, negm));
+          x1[e] = exp2_own(__fmaf_rn(s[bl * 16 + 8 + e], c, negm));
+        }
+        words[2 * bl] = encode8(x0, R);
+        words[2 * bl + 1] = encode8(x1, R);
+      }
+      uint8_t* pbuf = sP(sb);
+#pragma unroll
+      for (int q = 0; q < BC / 32; ++q)
+        *reinterpret_cast<uint4*>(pbuf + swz_offset(row, q, C::PROW)) =
+            make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+#pragma unroll
+      for (int kc = 0; kc < C::KP; ++kc)
+        *reinterpret_cast<uint32_t*>(sPsf(sb) + 512 * kc + sf_atom_offset(row, 0)) = sfw[kc];
+      fence_proxy_async_smem();
+      if (j > 0) {
+        ok = wait_all(o_bar, (j - 1) & 1, abort, p.status, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
+        tmem_wait_ld();
+        reg_fence(rr);
+        l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tbase + lrow + C::T_O + c0, o);
+            tmem_wait_ld();
+            reg_fence(o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
+            tmem_st32(tbase + lrow + C::T_O + c0, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[sb]);
+      alpha_prev = alpha;
+      m_run = mnew;
+    }
+    if (ok) ok = wait_all(o_bar, (nt - 1) & 1, abort, p.status, p.wait_ns);
+    if (ok) {
+      tc_fence_after();
+      uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
+      tmem_wait_ld();
+      reg_fence(rr);
+      l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
+      const float inv = (l_run > 0.0f) ? __frcp_rn(l_run) : 0.0f;
+      const long long orow = (long long)bh * p.N + qrow;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tbase + lrow + C::T_O + c0, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * i]), inv),
+                                                    __fmul_rn(__uint_as_float(o[2 * i + 1]), inv));
+          pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[c0 / 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      if (p.m_out) p.m_out[orow] = __float2half_rn(m_run);
+      if (p.l_out) p.l_out[orow] = __float2half_rn(l_run);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- single-tile probes
+
+// S = Q_hat K_hat^T of one 128 x BC tile through the same TMA / tcgen05.cp / MMA path as
+// the attention kernel (QK half only), written out as fp32 [128][BC].
+template <int D, int BC>
+__global__ void __launch_bounds__(128, 1)
+    k_probe_qk(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const uint8_t* qsf, const uint8_t* ksf, float* S, int* status, unsigned long long wait_ns) {
+  using C = AttnCfg<D, BC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + align_up(C::SZ_Q, 1024);
+  uint8_t* sQsf = sK + align_up(C::SZ_K, 1024);
+  uint8_t* sKsf = sQsf + C::SZ_QSF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKsf + C::SZ_KSF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 3);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[0], C::SZ_Q + C::SZ_K + C::SZ_QSF + C::SZ_KSF);
+    tma_load_2d(sQ, &tmQ, 0, 0, &bars[0]);
+    tma_load_2d(sK, &tmK, 0, 0, &bars[0]);
+    bulk_load(sQsf, qsf, C::SZ_QSF, &bars[0]);
+    bulk_load(sKsf, ksf, C::SZ_KSF, &bars[0]);
+  }
+  bool ok = wait_all(&bars[0], 0, abort, status, wait_ns);
+  if (ok && warp == 0) {
+    tc_fence_after();
+    if (lane == 0) {
+      const uint32_t T_SFQ = BC, T_SFK = BC + 4 * C::KQ;
+      for (int kc = 0; kc < C::KQ; ++kc) {
+        tmem_cp_sf_atom(tbase + T_SFQ + 4 * kc, sQsf + 512 * kc);
+        tmem_cp_sf_atom(tbase + T_SFK + 4 * kc, sKsf + 512 * kc);
+      }
+      for (int kc = 0; kc < C::KQ; ++kc)
+        mma_nvf4(tbase, smem_desc(smem_u32(sQ) + 32 * kc, 0, 8 * C::QROW, C::LQ),
+                 smem_desc(smem_u32(sK) + 32 * kc, 0, 8 * C::QROW, C::LQ), idesc_nvf4(128, BC),
+                 tbase + T_SFQ + 4 * kc, tbase + T_SFK + 4 * kc, kc > 0 ? 1u : 0u);
+      tc_commit(&bars[1]);
+    }
+    __syncwarp();
+  }
+  if (ok) ok = wait_all(&bars[1], 0, abort, status, wait_ns);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    for (int c0 = 0; c0 < BC; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + lrow + c0, r);
+      tmem_wait_ld();
+      reg_fence(r);
+      for (int i = 0; i < 32; ++i) S[(warp * 32 + lane) * BC + c0 + i] = __uint_as_float(r[i]);
+    }
+  } else if (threadIdx.x == 0) {
+    drain_wait(&bars[0], 0, status, wait_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// O = P_hat V_hat (fp32 [128][D]) and R = P_hat * ones (fp32 [128]) of one tile through
+// the attention kernel's PV path; P_hat arrives by TMA from a [128][BC/2] code tile.
+template <int D, int BC>
+__global__ void __launch_bounds__(128, 1)
+    k_probe_pv(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmV, const uint8_t* psf,
+               const uint8_t* vsf, float* O, float* Rout, int* status, unsigned long long wait_ns) {
+  using C = AttnCfg<D, BC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sP = smem;
+  uint8_t* sV = sP + align_up(C::SZ_P, 1024);
+  uint8_t* sOnes = sV + align_up(C::SZ_V, 1024);
+  uint8_t* sPsf = sOnes + align_up(C::SZ_ONES, 1024);
+  uint8_t* sVsf = sPsf + C::SZ_PSF;
+  uint8_t* s1sf = sVsf + C::SZ_VSF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s1sf + 512);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  volatile int* abort = reinterpret_cast<volatile int*>(bars + 3);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < (int)C::SZ_ONES / 4; i += 128) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
+  for (int i = threadIdx.x; i < 128; i += 128) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
+  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  constexpr uint32_t T_O = 0, T_R = D, T_SFP = D + 16, T_SFV = T_SFP + 4 * C::KP, T_SF1 = T_SFV + 4 * C::KP * C::NAV;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bars[0], C::SZ_P + C::SZ_V + C::SZ_PSF + C::SZ_VSF);
+    tma_load_2d(sP, &tmP, 0, 0, &bars[0]);
+    tma_load_2d(sV, &tmV, 0, 0, &bars[0]);
+    bulk_load(sPsf, psf, C::SZ_PSF, &bars[0]);
+    bulk_load(sVsf, vsf, C::SZ_VSF, &bars[0]);
+  }
+  bool ok = wait_all(&bars[0], 0, abort, status, wait_ns);
+  if (ok && warp == 0) {
+    tc_fence_after();
+    if (lane == 0) {
+      for (int i = 0; i < C::KP; ++i) tmem_cp_sf_atom(tbase + T_SFP + 4 * i, sPsf + 512 * i);
+      for (int i = 0; i < C::KP * C::NAV; ++i) tmem_cp_sf_atom(tbase + T_SFV + 4 * i, sVsf + 512 * i);
+      tmem_cp_sf_atom(tbase + T_SF1, s1sf);
+      for (int kc = 0; kc < C::KP; ++kc)
+        mma_nvf4(tbase + T_O, smem_desc(smem_u32(sP) + 32 * kc, 0, 8 * C::PROW, C::LP),
+                 smem_desc(smem_u32(sV) + 32 * kc, 0, 8 * C::PROW, C::LP), idesc_nvf4(128, D),
+                 tbase + T_SFP + 4 * kc, tbase + T_SFV + 4 * C::NAV * kc, kc > 0 ? 1u : 0u);
+      for (int kc = 0; kc < C::KP; ++kc)
+        mma_nvf4(tbase + T_R, smem_desc(smem_u32(sP) + 32 * kc, 0, 8 * C::PROW, C::LP),
+                 smem_desc(smem_u32(sOnes) + 32 * kc, 0, 8 * C::PROW, C::LP), idesc_nvf4(128, 16),
+                 tbase + T_SFP + 4 * kc, tbase + T_SF1, kc > 0 ? 1u : 0u);
+      tc_commit(&bars[1]);
+    }
+    __syncwarp();
+  }
+  if (ok) ok = wait_all(&bars[1], 0, abort, status, wait_ns);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t lrow = (uint32_t)(warp * 32) << 16;
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tbase + lrow + T_O + c0, r);
+      tmem_wait_ld();
+      reg_fence(r);
+      for (int i = 0; i < 32; ++i) O[(warp * 32 + lane) * D + c0 + i] = __uint_as_float(r[i]);
+    }
+    uint32_t rr[1] = {tmem_ld1(tbase + lrow + T_R)};
+    tmem_wait_ld();
+    reg_fence(rr);
+    Rout[warp * 32 + lane] = __uint_as_float(rr[0]);
+  } else if (threadIdx.x == 0) {
+    drain_wait(&bars[0], 0, status, wait_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+template <int D, int BC>
+constexpr uint32_t probe_qk_smem() {
+  using C = AttnCfg<D, BC>;
+  return align_up(C::SZ_Q, 1024) + align_up(C::SZ_K, 1024) + C::SZ_QSF + C::SZ_KSF + 64 + 1024;
+}
+template <int D, int BC>
+constexpr uint32_t probe_pv_smem() {
+  using C = AttnCfg<D, BC>;
+  return align_up(C::SZ_P, 1024) + align_up(C::SZ_V, 1024) + align_up(C::SZ_ONES, 1024) + C::SZ_PSF + C::SZ_VSF +
+         512 + 64 + 1024;
+}
+
+// Elementwise codec check: the device E2M1 / E4M3 conversions and the exp2 on given inputs.
+__global__ void k_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float* ex2) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float v = x[i];
+    e2m1[i] = (uint8_t)(cvt_e2m1x2(0.0f, v) & 0xF);
+    e4m3[i] = (uint8_t)cvt_e4m3(fabsf(v));
+    ex2[i] = exp2_own(v);
+  }
+}
+
+}  // namespace hifa4

@@ -1,0 +1,365 @@
+// Host side of the C ABI declared in include/hifa4.h: argument validation, tensor-map
+// construction, kernel dispatch over the supported (d, kv tile) shapes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/hifa4.h"
+#include "attn.cuh"
+#include "quant.cuh"
+
+using namespace hifa4;
+
+namespace {
+
+unsigned long long g_wait_ns = 2000000000ull;
+int g_inject = 0;
+
+bool device_ok() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  static std::vector<int> cache(64, -1);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 0 || dev >= 64) return false;
+  if (cache[dev] < 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cache[dev] = (major == 10 && minor == 0) ? 1 : 0;
+  }
+  return cache[dev] == 1;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+CUtensorMapSwizzle swizzle_of(int rowbytes) {
+  return rowbytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                        : rowbytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+}
+
+// 2-D byte tensor map: rows of `row_bytes` (stride `row_stride`), box of
+// `box_bytes` x `box_rows`, swizzled to match a K-major UMMA operand whose rows are
+// `box_bytes` long.
+bool make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint64_t row_stride,
+              uint32_t box_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_stride};
+  cuuint32_t box[2] = {box_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_of((int)box_bytes), CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool strides_ok(const void* base, const int64_t s[3]) {
+  if (!base || !s || !aligned16(base)) return false;
+  for (int i = 0; i < 3; ++i)
+    if (s[i] < 0 || (s[i] % 8) != 0) return false;
+  return true;
+}
+
+bool d_ok(int d) { return d == 64 || d == 128 || d == 256; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIFA4_OK : HIFA4_ERR_CUDA; }
+
+bool qt_ok(const hifa4_qtensor* t, int B, int H, int N, int d, int transposed) {
+  return t && t->codes && t->scales && aligned16(t->codes) && aligned16(t->scales) && t->B == B && t->H == H &&
+         t->N == N && t->d == d && t->transposed == transposed;
+}
+
+template <typename K>
+bool set_smem(K kernel, uint32_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+template <int D, int BC>
+int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
+                int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
+  using C = AttnCfg<D, BC>;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q->codes, D / 2, (uint64_t)B * Hq * N, D / 2, D / 2, 128) ||
+      !make_map(&tk, k->codes, D / 2, (uint64_t)B * Hkv * N, D / 2, D / 2, BC) ||
+      !make_map(&tv, vt->codes, N / 2, (uint64_t)B * Hkv * D, N / 2, BC / 2, D))
+    return HIFA4_ERR_CUDA;
+  // One CTA per SM when it holds all 512 TMEM columns: ask for more than half the SM's
+  // shared memory so a second CTA cannot become resident and block in tcgen05.alloc.
+  const uint32_t smem = (C::TMEM_COLS == 512 && C::SMEM < 120 * 1024) ? 120 * 1024 : C::SMEM;
+  static bool attr = set_smem(k_attn_fwd<D, BC>, smem);
+  if (!attr) return HIFA4_ERR_CUDA;
+  AttnParams p;
+  p.qsf = static_cast<const uint8_t*>(q->scales);
+  p.ksf = static_cast<const uint8_t*>(k->scales);
+  p.vsf = static_cast<const uint8_t*>(vt->scales);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.m_out = static_cast<__half*>(m_out);
+  p.l_out = static_cast<__half*>(l_out);
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.causal = causal ? 1 : 0;
+  p.c = (float)(1.4426950408889634074 / std::sqrt((double)D));
+  p.wait_ns = g_wait_ns;
+  p.inject = g_inject;
+  const unsigned grid = (unsigned)(B * Hq * (N / 128));
+  k_attn_fwd<D, BC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hifa4_status_string(int s) {
+  switch (s) {
+    case HIFA4_OK: return "HIFA4_OK";
+    case HIFA4_ERR_INVALID_ARG: return "HIFA4_ERR_INVALID_ARG";
+    case HIFA4_ERR_UNSUPPORTED_SHAPE: return "HIFA4_ERR_UNSUPPORTED_SHAPE";
+    case HIFA4_ERR_UNSUPPORTED_DEVICE: return "HIFA4_ERR_UNSUPPORTED_DEVICE";
+    case HIFA4_ERR_NONFINITE: return "HIFA4_ERR_NONFINITE";
+    case HIFA4_ERR_TIMEOUT: return "HIFA4_ERR_TIMEOUT";
+    case HIFA4_ERR_CUDA: return "HIFA4_ERR_CUDA";
+    default: return "HIFA4_ERR_UNKNOWN";
+  }
+}
+
+size_t hifa4_qtensor_codes_bytes(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  return (size_t)B * H * N * (d / 2);
+}
+
+size_t hifa4_qtensor_scales_bytes(int B, int H, int N, int d, int transposed) {
+  if (B <= 0 || H <= 0 || N <= 0 || d <= 0) return 0;
+  if (!transposed) return (size_t)B * H * (N / 128) * (d / 64) * 512;
+  return (size_t)B * H * (N / 64) * ((d + 127) / 128) * 512;
+}
+
+size_t hifa4_calibrate_workspace_bytes(int Hkv, int d) {
+  if (Hkv <= 0 || d <= 0) return 0;
+  return (size_t)2 * Hkv * d * sizeof(float);
+}
+
+int hifa4_calibrate_smooth(const void* q_cal, const void* k_cal, const int64_t q_strides[3],
+                           const int64_t k_strides[3], int B, int Hq, int Hkv, int N, int d, float alpha,
+                           float* s_out, float* sinv_out, void* workspace, cudaStream_t stream) {
+  if (!strides_ok(q_cal, q_strides) || !strides_ok(k_cal, k_strides) || !s_out || !sinv_out || !workspace ||
+      !(alpha >= 0.0f) || !std::isfinite(alpha))
+    return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || Hq % Hkv || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  float* amax = static_cast<float*>(workspace);
+  cudaError_t e = cudaMemsetAsync(amax, 0, hifa4_calibrate_workspace_bytes(Hkv, d), stream);
+  if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+  const int rows = 256;
+  AmaxArgs aq{static_cast<const __nv_bfloat16*>(q_cal), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, d, amax};
+  AmaxArgs ak{static_cast<const __nv_bfloat16*>(k_cal), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, d,
+              amax + Hkv * d};
+  k_channel_amax<<<dim3(B * Hq, (N + rows - 1) / rows), 128, 0, stream>>>(aq, rows);
+  k_channel_amax<<<dim3(B * Hkv, (N + rows - 1) / rows), 128, 0, stream>>>(ak, rows);
+  if (cudaGetLastError() != cudaSuccess) return HIFA4_ERR_CUDA;
+  std::vector<float> h(2 * (size_t)Hkv * d), s(Hkv * (size_t)d), si(Hkv * (size_t)d);
+  e = cudaMemcpyAsync(h.data(), amax, h.size() * sizeof(float), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+  for (size_t i = 0; i < s.size(); ++i) {
+    const float aq_ = h[i], ak_ = h[s.size() + i];
+    float v = 1.0f;
+    if (aq_ > 0.0f && ak_ > 0.0f) v = (float)std::pow((double)ak_ / (double)aq_, (double)alpha);
+    s[i] = v;
+    si[i] = 1.0f / v;
+  }
+  e = cudaMemcpyAsync(s_out, s.data(), s.size() * sizeof(float), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(sinv_out, si.data(), si.size() * sizeof(float), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  return cuda_status(e);
+}
+
+int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], const int64_t k_strides[3],
+                      int B, int Hq, int Hkv, int N, int d, const float* s, const float* sinv,
+                      const hifa4_qtensor* q_out, const hifa4_qtensor* k_out, int* status, cudaStream_t stream) {
+  if (!strides_ok(q, q_strides) || !strides_ok(k, k_strides) || !status || ((s == nullptr) != (sinv == nullptr)) ||
+      (s && (!aligned16(s) || !aligned16(sinv))))
+    return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0)) return HIFA4_ERR_INVALID_ARG;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
+                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / 128)};
+  QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
+                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / 128)};
+  const unsigned grid = (unsigned)(qa.tiles + ka.tiles);
+  switch (d) {
+    case 64: k_quant_rows<64><<<grid, 256, 0, stream>>>(qa, ka, status); break;
+    case 128: k_quant_rows<128><<<grid, 256, 0, stream>>>(qa, ka, status); break;
+    default: k_quant_rows<256><<<grid, 256, 0, stream>>>(qa, ka, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, int N, int d,
+                     const hifa4_qtensor* vt_out, int* status, cudaStream_t stream) {
+  if (!strides_ok(v, v_strides) || !status) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(vt_out, B, Hkv, N, d, 1)) return HIFA4_ERR_INVALID_ARG;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  QuantVtArgs a{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
+                static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales)};
+  const unsigned grid = (unsigned)(B * Hkv * (N / 64));
+  switch (d) {
+    case 64: k_quant_vt<64><<<grid, 128, 0, stream>>>(a, status); break;
+    case 128: k_quant_vt<128><<<grid, 128, 0, stream>>>(a, status); break;
+    default: k_quant_vt<256><<<grid, 256, 0, stream>>>(a, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
+                             int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
+                             void* l_out, int* status, cudaStream_t stream) {
+  if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
+    return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : 128;
+  if (kv_tile != 64 && kv_tile != 128) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q, B, Hq, N, d, 0) || !qt_ok(k, B, Hkv, N, d, 0) || !qt_ok(vt, B, Hkv, N, d, 1))
+    return HIFA4_ERR_INVALID_ARG;
+  if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  if (d == 64) {
+    return kv_tile == 64 ? launch_attn<64, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
+                         : launch_attn<64, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
+  } else if (d == 128) {
+    return kv_tile == 64 ? launch_attn<128, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
+                         : launch_attn<128, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
+  }
+  return launch_attn<256, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
+}
+
+size_t hifa4_attn_workspace_bytes(int B, int Hkv, int N, int d) {
+  const size_t c = hifa4_qtensor_codes_bytes(B, Hkv, N, d);
+  return ((c + 255) / 256) * 256 + hifa4_qtensor_scales_bytes(B, Hkv, N, d, 1);
+}
+
+int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v, const int64_t v_strides[3],
+                   int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* workspace,
+                   size_t workspace_bytes, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
+  if (!workspace || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || N <= 0 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < hifa4_attn_workspace_bytes(B, Hkv, N, d)) return HIFA4_ERR_INVALID_ARG;
+  const size_t c = hifa4_qtensor_codes_bytes(B, Hkv, N, d);
+  hifa4_qtensor vt;
+  vt.codes = workspace;
+  vt.scales = static_cast<uint8_t*>(workspace) + ((c + 255) / 256) * 256;
+  vt.B = B;
+  vt.H = Hkv;
+  vt.N = N;
+  vt.d = d;
+  vt.transposed = 1;
+  int r = hifa4_quantize_v(v, v_strides, B, Hkv, N, d, &vt, status, stream);
+  if (r != HIFA4_OK) return r;
+  return hifa4_attn_fwd_quantized(q, k, &vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream);
+}
+
+int hifa4_read_status(int* status, int clear, cudaStream_t stream) {
+  if (!status) return HIFA4_ERR_INVALID_ARG;
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, status, sizeof(int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && clear) {
+    e = cudaMemsetAsync(status, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  }
+  if (e != cudaSuccess) return HIFA4_ERR_CUDA;
+  if (h & ST_TIMEOUT) return HIFA4_ERR_TIMEOUT;
+  if (h & ST_NONFINITE) return HIFA4_ERR_NONFINITE;
+  return HIFA4_OK;
+}
+
+void hifa4_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns ? ns : 1; }
+void hifa4_debug_set_injection(int mode) { g_inject = mode; }
+
+int hifa4_probe_qk_tile(const void* q_codes, const void* q_scales, const void* k_codes, const void* k_scales, int d,
+                        int kv_tile, float* S, int* status, cudaStream_t stream) {
+  if (!q_codes || !q_scales || !k_codes || !k_scales || !S || !status || !aligned16(q_codes) || !aligned16(k_codes) ||
+      !aligned16(q_scales) || !aligned16(k_scales))
+    return HIFA4_ERR_INVALID_ARG;
+  if (!d_ok(d) || (kv_tile != 64 && kv_tile != 128)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, q_codes, d / 2, 128, d / 2, d / 2, 128) ||
+      !make_map(&tk, k_codes, d / 2, kv_tile, d / 2, d / 2, kv_tile))
+    return HIFA4_ERR_CUDA;
+  auto go = [&](auto kern, uint32_t smem) -> int {
+    if (!set_smem(kern, smem)) return HIFA4_ERR_CUDA;
+    kern<<<1, 128, smem, stream>>>(tq, tk, static_cast<const uint8_t*>(q_scales), static_cast<const uint8_t*>(k_scales),
+                                   S, status, g_wait_ns);
+    return cuda_status(cudaGetLastError());
+  };
+  if (d == 64) return kv_tile == 64 ? go(k_probe_qk<64, 64>, probe_qk_smem<64, 64>()) : go(k_probe_qk<64, 128>, probe_qk_smem<64, 128>());
+  if (d == 128) return kv_tile == 64 ? go(k_probe_qk<128, 64>, probe_qk_smem<128, 64>()) : go(k_probe_qk<128, 128>, probe_qk_smem<128, 128>());
+  return go(k_probe_qk<256, 64>, probe_qk_smem<256, 64>());
+}
+
+int hifa4_probe_pv_tile(const void* p_codes, const void* p_scales, const void* vt_codes, const void* vt_scales, int d,
+                        int kv_tile, float* O, float* R, int* status, cudaStream_t stream) {
+  if (!p_codes || !p_scales || !vt_codes || !vt_scales || !O || !R || !status || !aligned16(p_codes) ||
+      !aligned16(vt_codes) || !aligned16(p_scales) || !aligned16(vt_scales))
+    return HIFA4_ERR_INVALID_ARG;
+  if (!d_ok(d) || (kv_tile != 64 && kv_tile != 128)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  CUtensorMap tp, tv;
+  if (!make_map(&tp, p_codes, kv_tile / 2, 128, kv_tile / 2, kv_tile / 2, 128) ||
+      !make_map(&tv, vt_codes, kv_tile / 2, d, kv_tile / 2, kv_tile / 2, d))
+    return HIFA4_ERR_CUDA;
+  auto go = [&](auto kern, uint32_t smem) -> int {
+    if (!set_smem(kern, smem)) return HIFA4_ERR_CUDA;
+    kern<<<1, 128, smem, stream>>>(tp, tv, static_cast<const uint8_t*>(p_scales), static_cast<const uint8_t*>(vt_scales),
+                                   O, R, status, g_wait_ns);
+    return cuda_status(cudaGetLastError());
+  };
+  if (d == 64) return kv_tile == 64 ? go(k_probe_pv<64, 64>, probe_pv_smem<64, 64>()) : go(k_probe_pv<64, 128>, probe_pv_smem<64, 128>());
+  if (d == 128) return kv_tile == 64 ? go(k_probe_pv<128, 64>, probe_pv_smem<128, 64>()) : go(k_probe_pv<128, 128>, probe_pv_smem<128, 128>());
+  return go(k_probe_pv<256, 64>, probe_pv_smem<256, 64>());
+}
+
+int hifa4_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float* exp2_out, cudaStream_t stream) {
+  if (!x || !e2m1 || !e4m3 || !exp2_out || n < 0) return HIFA4_ERR_INVALID_ARG;
+  if (n == 0) return HIFA4_OK;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  const int grid = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+  k_probe_codec<<<grid, 256, 0, stream>>>(x, n, e2m1, e4m3, exp2_out);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

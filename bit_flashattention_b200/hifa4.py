@@ -1,0 +1,229 @@
+"""Thin Python binding of the C ABI in include/hifa4.h (argument marshalling only).
+
+Every step of the attention path runs in the CUDA library libhifa4.so; this module only
+allocates result tensors with torch (device memory), passes raw pointers and the current
+CUDA stream, and turns status codes into exceptions.  There is no CPU fallback: if the
+library is missing or the device is not an sm_100 GPU, calls raise.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhifa4.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "hifa4.h")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_NONFINITE, ERR_TIMEOUT, ERR_CUDA = range(7)
+
+
+class Hifa4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+class _QT(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("B", ctypes.c_int), ("H", ctypes.c_int),
+                ("N", ctypes.c_int), ("d", ctypes.c_int), ("transposed", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libhifa4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with bit_flashattention_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i, sz, f, ull = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_ulonglong
+        QP = ctypes.POINTER(_QT)
+        sig = {
+            "hifa4_status_string": ([i], ctypes.c_char_p),
+            "hifa4_qtensor_codes_bytes": ([i, i, i, i], sz),
+            "hifa4_qtensor_scales_bytes": ([i, i, i, i, i], sz),
+            "hifa4_calibrate_workspace_bytes": ([i, i], sz),
+            "hifa4_calibrate_smooth": ([P, P, P, P, i, i, i, i, i, f, P, P, P, P], i),
+            "hifa4_quantize_qk": ([P, P, P, P, i, i, i, i, i, P, P, QP, QP, P, P], i),
+            "hifa4_quantize_v": ([P, P, i, i, i, i, QP, P, P], i),
+            "hifa4_attn_fwd_quantized": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
+            "hifa4_attn_workspace_bytes": ([i, i, i, i], sz),
+            "hifa4_attn_fwd": ([QP, QP, P, P, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
+            "hifa4_read_status": ([P, i, P], i),
+            "hifa4_set_wait_limit_ns": ([ull], None),
+            "hifa4_debug_set_injection": ([i], None),
+            "hifa4_probe_qk_tile": ([P, P, P, P, i, i, P, P, P], i),
+            "hifa4_probe_pv_tile": ([P, P, P, P, i, i, P, P, P, P], i),
+            "hifa4_probe_codec": ([P, i, P, P, P, P], i),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions include/hifa4.h declares."""
+    txt = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"HIFA4_API\s+[\w\s\*]+?\b(hifa4_\w+)\s*\(", txt)))
+
+
+def status_string(code: int) -> str:
+    return lib().hifa4_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise Hifa4Error(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _strides(x):
+    s = x.stride()
+    if s[3] != 1:
+        raise ValueError("the channel dimension must be contiguous")
+    return (ctypes.c_int64 * 3)(s[0], s[1], s[2])
+
+
+class QTensor:
+    """A 4-bit tensor in the library's layout: uint8 `codes` and `scales` on the GPU."""
+
+    def __init__(self, B, H, N, d, transposed, device=None, codes=None, scales=None):
+        self.B, self.H, self.N, self.d, self.transposed = B, H, N, d, int(transposed)
+        L = lib()
+        nc = L.hifa4_qtensor_codes_bytes(B, H, N, d)
+        ns = L.hifa4_qtensor_scales_bytes(B, H, N, d, self.transposed)
+        self.codes = codes if codes is not None else torch.empty(nc, dtype=torch.uint8, device=device)
+        self.scales = scales if scales is not None else torch.empty(ns, dtype=torch.uint8, device=device)
+
+    def c(self):
+        return ctypes.byref(_QT(self.codes.data_ptr(), self.scales.data_ptr(), self.B, self.H, self.N, self.d,
+                                self.transposed))
+
+
+def new_status(device=None):
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def hifa4_read_status(status, clear=True):
+    return lib().hifa4_read_status(_ptr(status), int(clear), _stream())
+
+
+def hifa4_set_wait_limit_ns(ns: int):
+    lib().hifa4_set_wait_limit_ns(int(ns))
+
+
+def hifa4_debug_set_injection(mode: int):
+    lib().hifa4_debug_set_injection(int(mode))
+
+
+def hifa4_calibrate_smooth(q_cal, k_cal, alpha: float):
+    """Smooth-QK scales (s, s_inv), fp32 [Hkv, d] on q_cal's device.  Synchronises."""
+    B, Hq, N, d = q_cal.shape
+    Hkv = k_cal.shape[1]
+    dev = q_cal.device
+    s = torch.empty(Hkv, d, dtype=torch.float32, device=dev)
+    si = torch.empty_like(s)
+    ws = torch.empty(lib().hifa4_calibrate_workspace_bytes(Hkv, d), dtype=torch.uint8, device=dev)
+    _check(lib().hifa4_calibrate_smooth(_ptr(q_cal), _ptr(k_cal), _strides(q_cal), _strides(k_cal), B, Hq, Hkv, N, d,
+                                        float(alpha), _ptr(s), _ptr(si), _ptr(ws), _stream()), "hifa4_calibrate_smooth")
+    return s, si
+
+
+def hifa4_quantize_qk(q, k, s=None, sinv=None, status=None, out=None):
+    """Smooth-QK + 4-bit quantisation of bf16 Q [B,Hq,N,d] and K [B,Hkv,N,d] -> (QTensor, QTensor)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device))
+    st = status if status is not None else new_status(q.device)
+    _check(lib().hifa4_quantize_qk(_ptr(q), _ptr(k), _strides(q), _strides(k), B, Hq, Hkv, N, d, _ptr(s), _ptr(sinv),
+                                   out[0].c(), out[1].c(), _ptr(st), _stream()), "hifa4_quantize_qk")
+    return out
+
+
+def hifa4_quantize_v(v, status=None, out=None):
+    """4-bit quantisation of V^T (blocks of 16 tokens) of bf16 V [B,Hkv,N,d] -> QTensor."""
+    B, Hkv, N, d = v.shape
+    out = out if out is not None else QTensor(B, Hkv, N, d, 1, v.device)
+    st = status if status is not None else new_status(v.device)
+    _check(lib().hifa4_quantize_v(_ptr(v), _strides(v), B, Hkv, N, d, out.c(), _ptr(st), _stream()), "hifa4_quantize_v")
+    return out
+
+
+def _outputs(qq, dev, o, m, l):
+    B, Hq, N, d = qq.B, qq.H, qq.N, qq.d
+    if o is None:
+        o = torch.empty(B, Hq, N, d, dtype=torch.bfloat16, device=dev)
+    if m is None:
+        m = torch.empty(B, Hq, N, dtype=torch.float16, device=dev)
+    if l is None:
+        l = torch.empty(B, Hq, N, dtype=torch.float16, device=dev)
+    return o, m, l
+
+
+def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=None, m=None, l=None):
+    dev = qq.codes.device
+    o, m, l = _outputs(qq, dev, o, m, l)
+    st = status if status is not None else new_status(dev)
+    _check(lib().hifa4_attn_fwd_quantized(qq.c(), kq.c(), vt.c(), qq.B, qq.H, kq.H, qq.N, qq.d, int(causal),
+                                          int(kv_tile), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
+           "hifa4_attn_fwd_quantized")
+    return o, m, l
+
+
+def hifa4_attn_fwd(qq, kq, v, causal=True, kv_tile=0, status=None, workspace=None, o=None, m=None, l=None):
+    """Quantise V^T into a workspace and run the fused 4-bit attention -> (O bf16, m fp16, l fp16)."""
+    B, Hkv, N, d = v.shape
+    dev = v.device
+    o, m, l = _outputs(qq, dev, o, m, l)
+    need = lib().hifa4_attn_workspace_bytes(B, Hkv, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(lib().hifa4_attn_fwd(qq.c(), kq.c(), _ptr(v), _strides(v), qq.B, qq.H, Hkv, N, d, int(causal), int(kv_tile),
+                                _ptr(workspace), workspace.numel(), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
+           "hifa4_attn_fwd")
+    return o, m, l
+
+
+def hifa4_attn_workspace_bytes(B, Hkv, N, d):
+    return lib().hifa4_attn_workspace_bytes(B, Hkv, N, d)
+
+
+def hifa4_probe_qk_tile(q_codes, q_scales, k_codes, k_scales, d, kv_tile, status=None):
+    S = torch.empty(128, kv_tile, dtype=torch.float32, device=q_codes.device)
+    st = status if status is not None else new_status(q_codes.device)
+    _check(lib().hifa4_probe_qk_tile(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), d, kv_tile, _ptr(S),
+                                     _ptr(st), _stream()), "hifa4_probe_qk_tile")
+    return S
+
+
+def hifa4_probe_pv_tile(p_codes, p_scales, vt_codes, vt_scales, d, kv_tile, status=None):
+    O = torch.empty(128, d, dtype=torch.float32, device=p_codes.device)
+    R = torch.empty(128, dtype=torch.float32, device=p_codes.device)
+    st = status if status is not None else new_status(p_codes.device)
+    _check(lib().hifa4_probe_pv_tile(_ptr(p_codes), _ptr(p_scales), _ptr(vt_codes), _ptr(vt_scales), d, kv_tile, _ptr(O),
+                                     _ptr(R), _ptr(st), _stream()), "hifa4_probe_pv_tile")
+    return O, R
+
+
+def hifa4_probe_codec(x):
+    n = x.numel()
+    e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    ex = torch.empty(n, dtype=torch.float32, device=x.device)
+    _check(lib().hifa4_probe_codec(_ptr(x), n, _ptr(e2), _ptr(e4), _ptr(ex), _stream()), "hifa4_probe_codec")
+    return e2, e4, ex

@@ -1,0 +1,197 @@
+/*
+ * hifa4.h -- C ABI of a B200 (sm_100a) implementation of the HiFA4-style 4-bit
+ * FlashAttention forward pass.
+ *
+ * Method: "HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs for LLM
+ * Inference" (abstract).  Both QK^T and PV run as 4-bit GEMMs; the online-softmax state
+ * (running max m, normaliser l) is FP16; Smooth-QK rescales post-RoPE Q and K per channel
+ * (Q*s, K/s) with s fixed by an offline calibration; P-Reordering sums the normaliser
+ * from the same quantised weights P_hat that feed the PV GEMM, which lets the tensor core
+ * produce it (here: an extra MMA of P_hat against a block of ones).
+ *
+ * 4-bit format (the abstract does not give the HIF4 layout; this library states its own,
+ * NVFP4-style): E2M1 codes (two per byte, element 2i in the low nibble) with one unsigned
+ * E4M3 scale per 16 consecutive contraction elements.
+ *   scale = E4M3_RN(amax * RN(1/6));  code = E2M1_RN_satfinite(x * RN(1/scale)),
+ *   with 1/scale taken as 0 when scale == 0.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates or frees device memory.
+ *   - Work is enqueued on `stream` and is asynchronous, except where a function says it
+ *     synchronises.
+ *   - Return value: a hifa4_status.  Argument and shape errors are detected on the host
+ *     and nothing is launched.  Errors found on the device (non-finite input, a bounded
+ *     wait that ran out) are ORed as bits into a caller-provided device int `status`;
+ *     read them with hifa4_read_status().
+ *   - bf16 inputs [B, H, N, d] are addressed with element strides {b, h, n}; the channel
+ *     dimension must be contiguous, the base 16-byte aligned and every stride a multiple
+ *     of 8 elements.
+ *   - Shapes: d in {64, 128, 256}; Hq % Hkv == 0 (query head h uses kv head
+ *     h / (Hq/Hkv)); N % 128 == 0; N <= 63488 (the FP16 normaliser stays finite); causal
+ *     attention uses equal query and key lengths with key k visible to query i iff k <= i.
+ *   - Requires an sm_100 device (B200); anything else returns
+ *     HIFA4_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
+ */
+#ifndef HIFA4_H
+#define HIFA4_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define HIFA4_API __attribute__((visibility("default")))
+#else
+#define HIFA4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HIFA4_OK = 0,
+  HIFA4_ERR_INVALID_ARG = 1,       /* null pointer, bad stride or alignment, bad value */
+  HIFA4_ERR_UNSUPPORTED_SHAPE = 2, /* d, N, head counts or kv tile outside the supported set */
+  HIFA4_ERR_UNSUPPORTED_DEVICE = 3,/* current device is not sm_100 */
+  HIFA4_ERR_NONFINITE = 4,         /* a quantised input held inf or NaN (device-detected) */
+  HIFA4_ERR_TIMEOUT = 5,           /* a kernel's bounded wait ran out (device-detected) */
+  HIFA4_ERR_CUDA = 6               /* a CUDA runtime call or launch failed */
+} hifa4_status;
+
+/* Device status-word bits (ORed by kernels into the caller's `int* status`). */
+#define HIFA4_STATUS_NONFINITE 1
+#define HIFA4_STATUS_TIMEOUT 2
+
+/* Human-readable name of a status code; never NULL. */
+HIFA4_API const char* hifa4_status_string(int status);
+
+/*
+ * A 4-bit tensor in this library's layout (caller-owned device memory).
+ *   transposed == 0 (Q, K: blocks along d), logical [B, H, N, d]:
+ *     codes  [B][H][N][d/2]
+ *     scales [B][H][N/128][d/64][512]: per 128-row tile and 64-wide chunk of d, a
+ *            512-byte atom; row r (0..127), block s (0..3) of the chunk sits at byte
+ *            (r % 32) * 16 + (r / 32) * 4 + s.
+ *   transposed == 1 (V^T: blocks of 16 consecutive tokens per channel), logical
+ *   [B, H, d, N]:
+ *     codes  [B][H][d][N/2]
+ *     scales [B][H][N/64][ceil(d/128)][512]: per 64-token chunk and 128-channel group,
+ *            an atom as above with r = channel within the group (rows beyond d are 0).
+ * codes and scales must be 16-byte aligned.
+ */
+typedef struct {
+  void* codes;
+  void* scales;
+  int B, H, N, d;
+  int transposed;
+} hifa4_qtensor;
+
+/* Bytes of the codes / scales buffers of a 4-bit tensor with these logical sizes. */
+HIFA4_API size_t hifa4_qtensor_codes_bytes(int B, int H, int N, int d);
+HIFA4_API size_t hifa4_qtensor_scales_bytes(int B, int H, int N, int d, int transposed);
+
+/*
+ * Smooth-QK calibration (HiFA4 abstract: "calibration-static per-channel equivalent
+ * rescaling to Q and K after RoPE").  From a post-RoPE bf16 calibration sample Q_cal
+ * [B, Hq, N, d] and K_cal [B, Hkv, N, d]:
+ *   s[g, c]    = RN_fp32((amax_K[g, c] / amax_Q[g, c]) ^ alpha), computed in double
+ *                (s = 1 where either amax is 0; alpha = 0 gives s == 1),
+ *   s_inv[g,c] = RN_fp32(1 / s[g, c]),
+ * where amax_Q runs over the batch, the query heads of kv group g and all tokens, and
+ * amax_K over the batch and tokens of kv head g.  s_out and sinv_out are device fp32
+ * [Hkv * d].  `workspace` is device memory of hifa4_calibrate_workspace_bytes(Hkv, d)
+ * bytes.  N may be any positive value here.  SYNCHRONISES `stream` (it reads the channel
+ * maxima back to the host).  Offline step, not part of the timed path.
+ */
+HIFA4_API size_t hifa4_calibrate_workspace_bytes(int Hkv, int d);
+HIFA4_API int hifa4_calibrate_smooth(const void* q_cal, const void* k_cal, const int64_t q_strides[3],
+                           const int64_t k_strides[3], int B, int Hq, int Hkv, int N, int d, float alpha,
+                           float* s_out, float* sinv_out, void* workspace, cudaStream_t stream);
+
+/*
+ * Smooth-QK application + 4-bit quantisation of Q and K (one launch):
+ *   q' = RN(q * s[g(h), c]),  k' = RN(k * s_inv[g, c]),  then blocks of 16 along d.
+ * s and sinv are device fp32 [Hkv * d]; both NULL disables smoothing (s == 1).
+ * q_out / k_out: transposed == 0 tensors of sizes [B, Hq, N, d] / [B, Hkv, N, d].
+ * Sets HIFA4_STATUS_NONFINITE in *status if an input (after smoothing) is not finite.
+ */
+HIFA4_API int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], const int64_t k_strides[3],
+                      int B, int Hq, int Hkv, int N, int d, const float* s, const float* sinv,
+                      const hifa4_qtensor* q_out, const hifa4_qtensor* k_out, int* status, cudaStream_t stream);
+
+/*
+ * 4-bit quantisation of V^T: blocks of 16 consecutive tokens of one channel, no
+ * smoothing.  v: bf16 [B, Hkv, N, d]; vt_out: transposed == 1 tensor.
+ */
+HIFA4_API int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, int N, int d,
+                     const hifa4_qtensor* vt_out, int* status, cudaStream_t stream);
+
+/*
+ * The fused 4-bit attention forward on already quantised Q, K and V^T.
+ * For every (b, h, query row i), kv tiles j = 0, 1, ... of kv_tile keys (only tiles
+ * holding a visible key when causal):
+ *   S      = Q_hat K_hat_j^T                     (4-bit tensor-core MMA, fp32 accumulate)
+ *   m_new  = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e) / sqrt(d))
+ *   P      = E(RN(fma(S, c, -m_new)))            (E: the library's deterministic exp2)
+ *   P_hat  = 4-bit blocks of 16 keys, each block's scale from E(fma(blockmax S, c, -m_new))
+ *   alpha  = E(m - m_new)  (0 on the first tile)
+ *   O      = alpha * O + P_hat V_hat_j           (4-bit MMA)
+ *   r      = P_hat * 1                           (4-bit MMA against ones: P-Reordering)
+ *   l      = fp16_RN(fma(alpha, l, r)),  m = m_new
+ * and finally out = bf16_RN(O / l).  kv_tile is 64 or 128 (0 selects 128 for d <= 128 and
+ * 64 for d = 256; d = 256 supports only 64) and is part of the result's definition.
+ * o: bf16 [B, Hq, N, d] dense.  m_out, l_out: fp16 [B, Hq, N] dense, or NULL.
+ */
+HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
+                             int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
+                             void* l_out, int* status, cudaStream_t stream);
+
+/*
+ * The full attention forward on quantised Q, K and bf16 V: quantises V^T into
+ * `workspace` (hifa4_attn_workspace_bytes(B, Hkv, N, d) bytes of device memory, 16-byte
+ * aligned), then runs hifa4_attn_fwd_quantized.  Two launches on `stream`.
+ */
+HIFA4_API size_t hifa4_attn_workspace_bytes(int B, int Hkv, int N, int d);
+HIFA4_API int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v, const int64_t v_strides[3],
+                   int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* workspace,
+                   size_t workspace_bytes, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream);
+
+/*
+ * Synchronises `stream`, reads the device status word and maps it to a hifa4_status
+ * (TIMEOUT before NONFINITE before OK).  clear != 0 resets the word to 0 afterwards.
+ */
+HIFA4_API int hifa4_read_status(int* status, int clear, cudaStream_t stream);
+
+/* Wall-clock limit of every wait inside the kernels, in nanoseconds (default 2 s). */
+HIFA4_API void hifa4_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Test hook: mode 1 makes the attention kernel's loader skip kv tile 1, so its
+ * consumers' bounded waits run out and the call reports HIFA4_ERR_TIMEOUT through the
+ * status word without hanging.  0 (default) disables it.
+ */
+HIFA4_API void hifa4_debug_set_injection(int mode);
+
+/*
+ * Single-tile probes of the tensor-core path (test and debug exports).
+ *   hifa4_probe_qk_tile: S[128][kv_tile] fp32 = Q_hat K_hat^T for one 128-row Q tile
+ *     (codes [128][d/2], scale atoms d/64 x 512 B) and one kv_tile-row K tile (codes
+ *     [kv_tile][d/2], scale atoms d/64 x 512 B, keys in atom rows 0..kv_tile-1).
+ *   hifa4_probe_pv_tile: O[128][d] fp32 = P_hat V_hat and R[128] fp32 = P_hat * 1 for one
+ *     P_hat tile (codes [128][kv_tile/2], atoms kv_tile/64 x 512 B) and one V^T tile
+ *     (codes [d][kv_tile/2], atoms (kv_tile/64) x ceil(d/128) x 512 B).
+ *   hifa4_probe_codec: for each x[i]: E2M1 code of x, E4M3 code of |x| and the library's
+ *     exp2 E(x), computed by the device conversions the kernels use.
+ */
+HIFA4_API int hifa4_probe_qk_tile(const void* q_codes, const void* q_scales, const void* k_codes, const void* k_scales,
+                        int d, int kv_tile, float* S, int* status, cudaStream_t stream);
+HIFA4_API int hifa4_probe_pv_tile(const void* p_codes, const void* p_scales, const void* vt_codes, const void* vt_scales,
+                        int d, int kv_tile, float* O, float* R, int* status, cudaStream_t stream);
+HIFA4_API int hifa4_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float* exp2_out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HIFA4_H */

@@ -1,0 +1,77 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads without a GPU, exports
+every function include/hifa4.h declares, and its host-side validation rejects bad
+arguments before any device work."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from bit_flashattention_b200 import build, hifa4
+from tests import _layout
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return hifa4.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = hifa4.declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert hifa4.status_string(code).startswith("HIFA4_")
+    assert hifa4.status_string(99) == "HIFA4_ERR_UNKNOWN"
+
+
+def test_size_helpers(L):
+    assert L.hifa4_qtensor_codes_bytes(1, 32, 4096, 128) == 32 * 4096 * 64
+    assert L.hifa4_qtensor_scales_bytes(1, 32, 4096, 128, 0) == 32 * 4096 * 8
+    assert L.hifa4_qtensor_scales_bytes(1, 8, 4096, 128, 1) == 8 * 4096 * 8
+    assert L.hifa4_qtensor_scales_bytes(1, 8, 4096, 64, 1) == 8 * 64 * 512       # 64-channel atoms padded to 128
+    assert L.hifa4_attn_workspace_bytes(1, 8, 4096, 128) >= 8 * 128 * 2048 + 8 * 4096 * 8
+
+
+def test_host_validation_rejects_before_launch(L):
+    st = (ctypes.c_int64 * 3)(0, 0, 128)
+    qt = hifa4._QT(None, None, 1, 1, 128, 128, 0)
+    # null input
+    assert L.hifa4_quantize_qk(None, None, st, st, 1, 1, 1, 128, 128, None, None, ctypes.byref(qt),
+                               ctypes.byref(qt), None, None) == hifa4.ERR_INVALID_ARG
+    buf = np.zeros(4096, np.uint8)
+    p = ctypes.c_void_p(((buf.ctypes.data + 15) // 16) * 16)
+    status = ctypes.c_void_p(p.value + 2048)
+    # unsupported head dim / N not a multiple of 128
+    assert L.hifa4_quantize_v(p, st, 1, 1, 128, 96, ctypes.byref(qt), status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    assert L.hifa4_quantize_v(p, st, 1, 1, 100, 128, ctypes.byref(qt), status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    # misaligned stride
+    bad = (ctypes.c_int64 * 3)(0, 0, 129)
+    assert L.hifa4_quantize_v(p, bad, 1, 1, 128, 128, ctypes.byref(qt), status, None) == hifa4.ERR_INVALID_ARG
+    # d = 256 needs the 64-key tile
+    q = hifa4._QT(p, p, 1, 1, 128, 256, 0)
+    v = hifa4._QT(p, p, 1, 1, 128, 256, 1)
+    assert L.hifa4_attn_fwd_quantized(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v), 1, 1, 1, 128, 256, 1, 128,
+                                      p, None, None, status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    # GQA head counts must divide
+    assert L.hifa4_attn_fwd_quantized(ctypes.byref(q), ctypes.byref(q), ctypes.byref(v), 1, 3, 2, 128, 256, 1, 64,
+                                      p, None, None, status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+
+
+def test_layout_permutations_roundtrip():
+    rng = np.random.default_rng(0)
+    B, H, N, d = 2, 3, 256, 128
+    plain = rng.integers(0, 256, (B, H, N, d // 16), dtype=np.uint8)
+    at = _layout.rows_scales_from_plain(plain, B, H, N, d)
+    assert np.array_equal(_layout.rows_scales_to_plain(at, B, H, N, d), plain)
+    # the atom byte of row r, block s really is (r%32)*16 + (r//32)*4 + s
+    r, s = 77, 2
+    assert at[(r % 32) * 16 + (r // 32) * 4 + s] == plain[0, 0, r, s]
+    for dd in (64, 128, 256):
+        pv = rng.integers(0, 256, (B, H, dd, N // 16), dtype=np.uint8)
+        av = _layout.vt_scales_from_plain(pv, B, H, N, dd)
+        assert np.array_equal(_layout.vt_scales_to_plain(av, B, H, N, dd), pv)

@@ -126,7 +126,7 @@ def test_mirror_close_to_exact_attention(orc):
     # The 4-bit path stays close to fp64 softmax attention on the same dequantised Q, K, V
     # (numpy, no tiles): quantising P and keeping fp16 state add little on top of the
     # operand quantisation, while a dropped or misplaced term in the loop would not.
-    from test_oracle_quant import _dequant
+    from tests.test_oracle_quant import _dequant
     w = _small(Hq=4, Hkv=2, N=512, d=128)
     qz, (q, k, v) = _quantized(w)
     rows = np.arange(0, w.Hq * w.N)
