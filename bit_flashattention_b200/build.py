@@ -5,7 +5,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "hifa4_api.cu")
+SRCS = [os.path.join(HERE, "csrc", f) for f in ("hifa4_api.cu", "hifa4_noalloc.cu")]
 DEPS = [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "method.cuh", "quant.cuh", "attn.cuh")] + \
        [os.path.join(ROOT, "include", "hifa4.h")]
 LIB = os.path.join(HERE, "libhifa4.so")
@@ -28,10 +28,10 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    newest = max(os.path.getmtime(p) for p in [SRC] + DEPS)
+    newest = max(os.path.getmtime(p) for p in SRCS + DEPS)
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
         return LIB
-    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", LIB, SRC]
+    cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-o", LIB] + SRCS
     subprocess.check_call(cmd)
     return LIB
 

@@ -159,6 +159,25 @@ HIFA4_API int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, con
                    size_t workspace_bytes, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream);
 
 /*
+ * hifa4_attn_fwd without a caller workspace (the method's pages have no counterpart of
+ * this entry point; it exists for callers that cannot allocate device memory -- e.g. a
+ * serving process whose device memory is all handed out up front, or a latency-critical
+ * loop that must not block on cudaMalloc).  Same arguments and results as
+ * hifa4_attn_fwd minus the workspace: the 4-bit V^T goes to a 16 MiB scratch array
+ * compiled into the library, which every GPU that loads the library holds until the
+ * process exits.  Workloads whose hifa4_attn_workspace_bytes(B, Hkv, N, d) exceeds
+ * 16 MiB are rejected with HIFA4_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ * Allocates nothing.  The first call on a device looks up the scratch array's device
+ * address (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls on a device share the scratch: calls whose GPU work may overlap (e.g. on
+ * unordered streams) race on it.
+ */
+HIFA4_API int hifa4_attn_fwd_noalloc(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v,
+                                     const int64_t v_strides[3], int B, int Hq, int Hkv, int N, int d, int causal,
+                                     int kv_tile, void* o, void* m_out, void* l_out, int* status,
+                                     cudaStream_t stream);
+
+/*
  * Synchronises `stream`, reads the device status word and maps it to a hifa4_status
  * (TIMEOUT before NONFINITE before OK).  clear != 0 resets the word to 0 afterwards.
  */
