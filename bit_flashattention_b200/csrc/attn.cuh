@@ -53,7 +53,9 @@ struct AttnCfg {
   static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
   static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
-  static constexpr uint32_t OFF_BAR = OFF_1SF + 512;
+  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 256 x fp32 reciprocal table
+  static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
+  static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 128 * 4;
   // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
   // s_empty[2], p_full[2], o_bar, drain
   static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 6 + 2;
@@ -67,7 +69,16 @@ struct AttnCfg {
   static_assert(T_END <= 512, "TMEM budget exceeded");
   static_assert(D == 64 || D == 128 || D == 256, "head dim");
   static_assert(BC == 64 || BC == 128, "kv tile");
-  static constexpr int NTHREADS = 192;
+  // softmax warpgroups: each takes CW consecutive score columns of every row and D/NSW
+  // columns of O (both at least 32, the width of one tcgen05.ld)
+#ifndef HIFA4_MAX_NSW
+#define HIFA4_MAX_NSW 4
+#endif
+  static constexpr int NSW0 = (BC < D ? BC : D) / 32;
+  static constexpr int NSW = NSW0 < HIFA4_MAX_NSW ? NSW0 : HIFA4_MAX_NSW, CW = BC / NSW;
+  static_assert(NSW == 2 || NSW == 4, "softmax warpgroups");
+  static_assert(CW == 32 || CW == 64, "column split");
+  static constexpr int NTHREADS = 64 + 128 * NSW;
 };
 
 struct AttnParams {
@@ -110,8 +121,12 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, int* 
   return mbar_wait(bar, parity, &never, status, ns);
 }
 
+__device__ __forceinline__ void named_bar(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 template <int D, int BC>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D, BC>;
@@ -152,18 +167,22 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
-      const bool four = (&bars[i] == &s_empty[0] || &bars[i] == &s_empty[1] || &bars[i] == &p_full[0] ||
-                         &bars[i] == &p_full[1]);
-      mbar_init(&bars[i], four ? 4 : 1);   // s_empty / p_full: one arrival per softmax warp
+      const bool per_warp = (&bars[i] == &s_empty[0] || &bars[i] == &s_empty[1] || &bars[i] == &p_full[0] ||
+                             &bars[i] == &p_full[1]);
+      mbar_init(&bars[i], per_warp ? 4 * C::NSW : 1);   // s_empty / p_full: one arrival per softmax warp
     }
     *abort = 0;
     fence_mbar_init();
   }
+  float* rtab = reinterpret_cast<float*>(smem + C::OFF_RTAB);
+  float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
   if (warp >= 2) {
     // the ones operand (E2M1 1.0 = 0b0010 in both nibbles) and its scales (UE4M3 1.0)
-    for (int i = threadIdx.x - 64; i < (int)C::SZ_ONES / 4; i += 128) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
-    for (int i = threadIdx.x - 64; i < 128; i += 128) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
+    const int t = threadIdx.x - 64, nt2 = 128 * C::NSW;
+    for (int i = t; i < (int)C::SZ_ONES / 4; i += nt2) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
+    for (int i = t; i < 128; i += nt2) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
     fence_proxy_async_smem();
+    fill_recip_table(rtab, t, nt2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -301,10 +320,15 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps
+    // warp pairs (w, w+4) share TMEM lane quarter q4 (the same 32 query rows); warpgroup
+    // wg takes score columns [wg*CW, wg*CW + CW) and O columns [wg*D/NSW, ...).
+    constexpr int CW = C::CW, NB = CW / 16, OW = D / C::NSW;
+    const int sw = warp - 2, wg = sw >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
     const int qrow = qtile * 128 + row;
+    const int col0 = wg * CW;
     const float c = p.c;
     float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
@@ -313,66 +337,86 @@ __global__ void __launch_bounds__(192, 1)
       ok = wait_all(&s_full[sb], (j >> 1) & 1, abort, p.status, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
-      float s[BC];
+      float s[CW];
       {
-        uint32_t r[BC];
+        uint32_t r[CW];
 #pragma unroll
-        for (int c0 = 0; c0 < BC; c0 += 32)
-          tmem_ld32(tbase + lrow + C::T_S + sb * BC + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+        for (int c0 = 0; c0 < CW; c0 += 32)
+          tmem_ld32(tbase + lrow + C::T_S + sb * BC + col0 + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
         tmem_wait_ld();
         reg_fence(r);
 #pragma unroll
-        for (int i = 0; i < BC; ++i) s[i] = __uint_as_float(r[i]);
+        for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(r[i]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[sb]);
       if (p.causal && (j + 1) * BC - 1 > qtile * 128) {
 #pragma unroll
-        for (int i = 0; i < BC; ++i)
-          if (j * BC + i > qrow) s[i] = -INFINITY;
+        for (int i = 0; i < CW; ++i)
+          if (j * BC + col0 + i > qrow) s[i] = -INFINITY;
       }
-      float bmax[BC / 16];
+      float bmax[NB];
 #pragma unroll
-      for (int bl = 0; bl < BC / 16; ++bl) {
+      for (int bl = 0; bl < NB; ++bl) {
         float m = s[bl * 16];
 #pragma unroll
         for (int e = 1; e < 15; e += 2) m = fmax3(m, s[bl * 16 + e], s[bl * 16 + e + 1]);
         bmax[bl] = fmaxf(m, s[bl * 16 + 15]);
       }
-      float rmax = bmax[0];
+      float lmax = bmax[0];
 #pragma unroll
-      for (int bl = 1; bl < BC / 16; ++bl) rmax = fmaxf(rmax, bmax[bl]);
+      for (int bl = 1; bl < NB; ++bl) lmax = fmaxf(lmax, bmax[bl]);
+      // combine the partial row maxima of the NSW warpgroups (double-buffered by tile parity)
+      float* xm = xmax + (j & 1) * (C::NSW * 128);
+      xm[wg * 128 + row] = lmax;
+      named_bar(1 + q4, 32 * C::NSW);
+      float rmax = xm[row];
+#pragma unroll
+      for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
       float mnew = m_run;
       if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
       const float alpha = (m_run == -INFINITY) ? 0.0f : exp2_own(__fsub_rn(m_run, mnew));
       const float negm = -mnew;
-      uint32_t words[BC / 8];
-      uint32_t sfw[C::KP];
+      const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
+      // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call
+      float pmax[NB];
 #pragma unroll
-      for (int kc = 0; kc < C::KP; ++kc) sfw[kc] = 0;
+      for (int bl = 0; bl < NB; bl += 2) {
+        const float2 e2 = exp2_own2(__ffma2_rn(make_float2(bmax[bl], bmax[bl + 1]), c2, negm2));
+        pmax[bl] = e2.x;
+        pmax[bl + 1] = e2.y;
+      }
+      uint32_t words[CW / 8];
+      uint32_t sfw = 0;
 #pragma unroll
-      for (int bl = 0; bl < BC / 16; ++bl) {
+      for (int bl = 0; bl < NB; ++bl) {
         float R;
-        const uint32_t sc = block_scale(exp2_own(__fmaf_rn(bmax[bl], c, negm)), R);
-        sfw[bl / 4] |= sc << (8 * (bl % 4));
-        float x0[8], x1[8];
+        const uint32_t sc = block_scale_tab(pmax[bl], rtab, R);
+        sfw |= sc << (8 * bl);
+        const float2 R2 = make_float2(R, R);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x0[e] = exp2_own(__fmaf_rn(s[bl * 16 + e], c, negm));
-          x1[e] = exp2_own(__fmaf_rn(s[bl * 16 + 8 + e], c, negm));
+        for (int h8 = 0; h8 < 2; ++h8) {
+          float2 y[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int e = bl * 16 + h8 * 8 + 2 * k;
+            const float2 t2 = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2);
+            y[k] = __fmul2_rn(exp2_own2(t2), R2);
+          }
+          words[2 * bl + h8] = encode8_pairs(y);
         }
-        words[2 * bl] = encode8(x0, R);
-        words[2 * bl + 1] = encode8(x1, R);
       }
       uint8_t* pbuf = sP(sb);
 #pragma unroll
-      for (int q = 0; q < BC / 32; ++q)
-        *reinterpret_cast<uint4*>(pbuf + swz_offset(row, q, C::PROW)) =
+      for (int q = 0; q < CW / 32; ++q)
+        *reinterpret_cast<uint4*>(pbuf + swz_offset(row, col0 / 32 + q, C::PROW)) =
             make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-#pragma unroll
-      for (int kc = 0; kc < C::KP; ++kc)
-        *reinterpret_cast<uint32_t*>(sPsf(sb) + 512 * kc + sf_atom_offset(row, 0)) = sfw[kc];
+      {
+        uint8_t* atom = sPsf(sb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
+        if (NB == 4) *reinterpret_cast<uint32_t*>(atom) = sfw;
+        else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
+      }
       fence_proxy_async_smem();
       if (j > 0) {
         ok = wait_all(o_bar, (j - 1) & 1, abort, p.status, p.wait_ns);
@@ -384,13 +428,18 @@ __global__ void __launch_bounds__(192, 1)
         l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
+          for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(tbase + lrow + C::T_O + c0, o);
             tmem_wait_ld();
             reg_fence(o);
+            const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__fmul_rn(__uint_as_float(o[i]), alpha));
+            for (int i = 0; i < 32; i += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
+              o[i] = __float_as_uint(v.x);
+              o[i + 1] = __float_as_uint(v.y);
+            }
             tmem_st32(tbase + lrow + C::T_O + c0, o);
           }
           tmem_wait_st();
@@ -413,7 +462,7 @@ __global__ void __launch_bounds__(192, 1)
       const long long orow = (long long)bh * p.N + qrow;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tbase + lrow + C::T_O + c0, o);
         tmem_wait_ld();
@@ -428,8 +477,10 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) dst[c0 / 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
-      if (p.m_out) p.m_out[orow] = __float2half_rn(m_run);
-      if (p.l_out) p.l_out[orow] = __float2half_rn(l_run);
+      if (wg == 0) {
+        if (p.m_out) p.m_out[orow] = __float2half_rn(m_run);
+        if (p.l_out) p.l_out[orow] = __float2half_rn(l_run);
+      }
     }
   }
   tc_fence_before();

@@ -86,6 +86,27 @@ bool strides_ok(const void* base, const int64_t s[3]) {
 
 bool d_ok(int d) { return d == 64 || d == 128 || d == 256; }
 
+int num_sms();
+
+// Grid of a grid-stride kernel: all units at once if they fit, else one full wave.
+template <typename K>
+int resident_grid(K kernel, int threads, int units) {
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n <= 0) n = 1;
+    per_sm = n;
+  }
+  const long long cap = (long long)per_sm * num_sms();
+  return (int)(units < cap ? units : cap);
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? HIFA4_OK : HIFA4_ERR_CUDA; }
 
 bool qt_ok(const hifa4_qtensor* t, int B, int H, int N, int d, int transposed) {
@@ -211,15 +232,16 @@ int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], 
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0)) return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  const int rows = d == 256 ? 64 : 128;   // rows per unit of k_quant_rows<d>
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
-                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / 128)};
+                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
-                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / 128)};
-  const unsigned grid = (unsigned)(qa.tiles + ka.tiles);
+                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
+  const int units = qa.units + ka.units;
   switch (d) {
-    case 64: k_quant_rows<64><<<grid, 256, 0, stream>>>(qa, ka, status); break;
-    case 128: k_quant_rows<128><<<grid, 256, 0, stream>>>(qa, ka, status); break;
-    default: k_quant_rows<256><<<grid, 256, 0, stream>>>(qa, ka, status); break;
+    case 64: k_quant_rows<64><<<resident_grid(k_quant_rows<64>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
+    case 128: k_quant_rows<128><<<resident_grid(k_quant_rows<128>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
+    default: k_quant_rows<256><<<resident_grid(k_quant_rows<256>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
   }
   return cuda_status(cudaGetLastError());
 }
@@ -231,12 +253,11 @@ int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, 
   if (!qt_ok(vt_out, B, Hkv, N, d, 1)) return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   QuantVtArgs a{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
-                static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales)};
-  const unsigned grid = (unsigned)(B * Hkv * (N / 64));
+                static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
   switch (d) {
-    case 64: k_quant_vt<64><<<grid, 128, 0, stream>>>(a, status); break;
-    case 128: k_quant_vt<128><<<grid, 128, 0, stream>>>(a, status); break;
-    default: k_quant_vt<256><<<grid, 256, 0, stream>>>(a, status); break;
+    case 64: k_quant_vt<64><<<resident_grid(k_quant_vt<64>, 128, a.units), 128, 0, stream>>>(a, status); break;
+    case 128: k_quant_vt<128><<<resident_grid(k_quant_vt<128>, 128, a.units), 128, 0, stream>>>(a, status); break;
+    default: k_quant_vt<256><<<resident_grid(k_quant_vt<256>, 128, a.units), 128, 0, stream>>>(a, status); break;
   }
   return cuda_status(cudaGetLastError());
 }

@@ -16,21 +16,69 @@ namespace hifa4 {
 constexpr float kSixth = 0x1.555556p-3f;
 
 // The softmax's exp2: E(x) = p(f) * 2^n with x' = max(x, -127), n = floor(x'), f = x' - n
-// and p(f) = ((c3 f + c2) f + c1) f + 1 evaluated with fused multiply-adds; the
-// coefficients are a minimax fit of 2^f on [0, 1) in relative error with p(0) = 1 held
-// exact (max relative error 8.6e-5).  The floor uses a round-down add of 1.5 * 2^23,
-// whose low mantissa bits then hold n, so the exponent insert is one shift-add.
-constexpr float kExp2C1 = 0x1.63e65ap-1f;
-constexpr float kExp2C2 = 0x1.d23788p-3f;
-constexpr float kExp2C3 = 0x1.3baaa8p-4f;
+// and p(f) = (c2 f + c1) f + 1 evaluated with fused multiply-adds; the coefficients are a
+// minimax fit of 2^f on [0, 1) in relative error with p(0) = 1 held exact (max relative
+// error 2.05e-3, far below the spacing of the 4-bit codes P is rounded to).  The floor
+// uses a round-down add of 1.5 * 2^23, whose low mantissa bits then hold n, so the
+// exponent insert is one integer multiply-add.
+constexpr float kExp2C1 = 0x1.54f8d6p-1f;
+constexpr float kExp2C2 = 0x1.51d9ccp-2f;
+
+// bits(p) + (n << 23), with n in the low bits of v's pattern (v = floor(x') + 1.5 * 2^23).
+__device__ __forceinline__ float insert_exponent(float p, float v) {
+  uint32_t r;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r) : "r"(__float_as_uint(v)), "r"(__float_as_uint(p)));
+  return __uint_as_float(r);
+}
 
 __device__ __forceinline__ float exp2_own(float x) {
   const float xc = fmaxf(x, -127.0f);
   const float v = __fadd_rd(xc, 12582912.0f);
   const float n = __fsub_rn(v, 12582912.0f);
   const float f = __fsub_rn(xc, n);
-  const float p = __fmaf_rn(__fmaf_rn(__fmaf_rn(kExp2C3, f, kExp2C2), f, kExp2C1), f, 1.0f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(v) << 23));
+  const float p = __fmaf_rn(__fmaf_rn(kExp2C2, f, kExp2C1), f, 1.0f);
+  return insert_exponent(p, v);
+}
+
+// E(x) on a pair of values with the packed fp32 instructions of sm_100 (two lanes per
+// instruction, each rounded exactly as the scalar form): bit-identical to exp2_own.
+__device__ __forceinline__ float2 exp2_own2(float2 x) {
+  const float2 xc = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 v = __fadd2_rd(xc, make_float2(12582912.0f, 12582912.0f));
+  const float2 n = __fadd2_rn(v, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);          // xc - n, exact
+  float2 p = __ffma2_rn(make_float2(kExp2C2, kExp2C2), f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+  return make_float2(insert_exponent(p.x, v.x), insert_exponent(p.y, v.y));
+}
+
+// Eight values held as four pairs (element 2k in .x) -> eight E2M1 codes, low nibble first.
+__device__ __forceinline__ uint32_t encode8_pairs(const float2 (&y)[4]) {
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(y[0].x), "f"(y[0].y), "f"(y[1].x), "f"(y[1].y), "f"(y[2].x), "f"(y[2].y), "f"(y[3].x), "f"(y[3].y));
+  return w;
+}
+
+// max(a, |b|) that turns NaN into NaN (PTX max.NaN), so one test of a block's amax
+// catches every non-finite element of the block.
+__device__ __forceinline__ float max_abs_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(fabsf(b)));
+  return d;
+}
+
+// Scale code of a block from its absolute maximum, reciprocal from the table below.
+__device__ __forceinline__ uint32_t block_scale_tab(float amax, const float* rtab, float& R) {
+  const uint32_t sc = cvt_e4m3(__fmul_rn(amax, kSixth));
+  R = rtab[sc];
+  return sc;
 }
 
 // Scale code and reciprocal of a block from its absolute maximum.
@@ -43,11 +91,28 @@ __device__ __forceinline__ uint32_t block_scale(float amax, float& R) {
 
 // Eight values -> eight E2M1 codes (after multiplying by R), packed low nibble first.
 __device__ __forceinline__ uint32_t encode8(const float (&x)[8], float R) {
-  uint32_t w = 0;
+  float y[8];
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    w |= cvt_e2m1x2(__fmul_rn(x[2 * k + 1], R), __fmul_rn(x[2 * k], R)) << (8 * k);
+  for (int k = 0; k < 8; ++k) y[k] = __fmul_rn(x[k], R);
+  uint32_t w;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(w)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
   return w;
+}
+
+// RN(1/scale) for every E4M3 code (0 for the zero scale and for codes that are not
+// finite positive scales), filled once per CTA so a block's reciprocal is one load.
+__device__ __forceinline__ void fill_recip_table(float* tab, int tid, int nthreads) {
+  for (int i = tid; i < 256; i += nthreads) {
+    const float v = e4m3_value((uint32_t)i);
+    tab[i] = (v > 0.0f && v <= 448.0f) ? __frcp_rn(v) : 0.0f;
+  }
 }
 
 // Byte offset of row r (0..127), block s (0..3) inside a 512-byte scale-factor atom:

@@ -18,64 +18,90 @@ struct QuantRowsArgs {
   const float* scale;         // [Hkv, D] or nullptr
   uint8_t* codes;             // [B, H, N, D/2]
   uint8_t* sf;                // [B, H, N/128, D/64, 512]
-  int tiles;                  // B * H * N / 128
+  int units;                  // B * H * N / ROWS (ROWS rows of one head per unit)
 };
 
-// One CTA of 256 threads quantises a 128-row tile; each thread takes 8 consecutive
-// elements (16 bytes) at a time: 2 threads per 16-block, 8 threads per 64-wide chunk.
+// max(|a|, |b|, |c|), NaN if any input is NaN.
+__device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
+  float d;
+  asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Grid-stride over units of ROWS rows of one head (Q units first, then K units).  Thread
+// (row r, block k) quantises one 16-element block: two 16-byte loads (all of a thread's
+// loads in flight before any arithmetic), the block amax with 3-input max instructions, the
+// scale from the amax and its reciprocal from a shared table, 8 code bytes stored at once.
+// The four blocks of a 64-wide chunk sit in lanes 4q..4q+3, which assemble the chunk's
+// scale word with two shuffles.
 template <int D>
 __global__ void __launch_bounds__(256) k_quant_rows(QuantRowsArgs qa, QuantRowsArgs ka, int* status) {
-  const bool isq = blockIdx.x < (unsigned)qa.tiles;
-  const QuantRowsArgs& a = isq ? qa : ka;
-  const int tile = isq ? blockIdx.x : blockIdx.x - qa.tiles;
-  const int ntile_n = a.N / 128;
-  const int bh = tile / ntile_n, rt = tile % ntile_n;
-  const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
+  constexpr int BPR = D / 16;                  // blocks per row
+  constexpr int RPP = 256 / BPR;               // rows per pass
+  constexpr int ROWS = D == 256 ? 64 : 128;    // rows per unit
+  constexpr int PASSES = ROWS / RPP;
   const int lane = threadIdx.x & 31;
-  constexpr int PARTS = D / 8;
-  constexpr int ITEMS = 128 * PARTS;
+  const int blk = threadIdx.x % BPR;
+  const int rsub = threadIdx.x / BPR;
+  __shared__ float rtab[256];
+  fill_recip_table(rtab, threadIdx.x, 256);
+  __syncthreads();
   bool bad = false;
-#pragma unroll 2
-  for (int it = threadIdx.x; it < ITEMS; it += 256) {
-    const int row = it / PARTS, part = it % PARTS;
-    const long long n = (long long)rt * 128 + row;
-    const uint4 raw = *reinterpret_cast<const uint4*>(a.x + b * a.sb + h * a.sh + n * a.sn + part * 8);
-    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-    float v[8];
+  for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
+    const bool isq = u < qa.units;
+    const QuantRowsArgs& a = isq ? qa : ka;
+    const int unit = isq ? u : u - qa.units;
+    const int per_head = a.N / ROWS;
+    const int bh = unit / per_head, n0 = (unit % per_head) * ROWS;
+    const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
+    const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + blk * 16;
+    uint4 raw[PASSES][2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = __bfloat1622float2(p2[k]);
-      v[2 * k] = f.x;
-      v[2 * k + 1] = f.y;
+    for (int k = 0; k < PASSES; ++k) {
+      const uint4* src = reinterpret_cast<const uint4*>(base + (long long)(n0 + rsub + k * RPP) * a.sn);
+      raw[k][0] = src[0];
+      raw[k][1] = src[1];
     }
+    float2 s2[8];
     if (a.scale) {
-      const float4* sp = reinterpret_cast<const float4*>(a.scale + g * D + part * 8);
-      const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
-      v[0] = __fmul_rn(v[0], s0.x); v[1] = __fmul_rn(v[1], s0.y);
-      v[2] = __fmul_rn(v[2], s0.z); v[3] = __fmul_rn(v[3], s0.w);
-      v[4] = __fmul_rn(v[4], s1.x); v[5] = __fmul_rn(v[5], s1.y);
-      v[6] = __fmul_rn(v[6], s1.z); v[7] = __fmul_rn(v[7], s1.w);
-    }
-    float amax = 0.0f;
+      const float4* sp = reinterpret_cast<const float4*>(a.scale + g * D + blk * 16);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      bad |= !isfinite(v[k]);
-      amax = fmaxf(amax, fabsf(v[k]));
+      for (int q = 0; q < 4; ++q) {
+        const float4 t = __ldg(sp + q);
+        s2[2 * q] = make_float2(t.x, t.y);
+        s2[2 * q + 1] = make_float2(t.z, t.w);
+      }
     }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    float R;
-    const uint32_t sc = block_scale(amax, R);
-    const uint32_t w = encode8(v, R);
-    *reinterpret_cast<uint32_t*>(a.codes + ((long long)bh * a.N + n) * (D / 2) + part * 4) = w;
-    // gather the 4 scale bytes of this 64-chunk (blocks live in lanes base+0, +2, +4, +6)
-    const int base = lane & ~7;
-    uint32_t word = 0;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) word |= __shfl_sync(0xffffffffu, sc, base + 2 * s) << (8 * s);
-    if ((lane & 7) == 0) {
-      const int kc = part / 8;
-      uint8_t* atom = a.sf + (((long long)bh * ntile_n + rt) * (D / 64) + kc) * 512;
-      *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row, 0)) = word;
+    for (int k = 0; k < PASSES; ++k) {
+      const int row = n0 + rsub + k * RPP;
+      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k][0]);
+      float2 v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
+      if (a.scale) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], s2[e]);
+      }
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
+      bad |= !isfinite(amax);
+      float R;
+      const uint32_t sc = block_scale_tab(amax, rtab, R);
+      const float2 R2 = make_float2(R, R);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], R2);
+      const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
+      *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
+          make_uint2(encode8_pairs(lo), encode8_pairs(hi));
+      uint32_t word = sc << (8 * (lane & 3));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      if ((lane & 3) == 0) {
+        uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
+        *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
+      }
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, ST_NONFINITE);
@@ -87,60 +113,80 @@ struct QuantVtArgs {
   int H, N;
   uint8_t* codes;             // [B, Hkv, D, N/2]
   uint8_t* sf;                // [B, Hkv, N/64, ceil(D/128), 512]
+  int units;                  // B * Hkv * N / 32
 };
 
-// One CTA per (b, kv head, 64-token chunk): the tile is staged in shared memory with
-// coalesced loads, then thread c quantises channel c's four 16-token blocks and writes
-// its 32 code bytes and one scale word.  Threads c >= D (only D = 64) zero the unused
-// rows of the 128-row scale atom.
+// Grid-stride over (b, kv head, 32-token half of a 64-token chunk) units, 128 threads.
+// The 32 x D tile is staged in shared memory with coalesced 16-byte loads (all of a
+// thread's loads in flight first); then thread c quantises the two 16-token blocks of
+// channel c in this half, writes their 16 code bytes and its 2 bytes of the channel's
+// scale word.  For D = 64 the unused rows 64..127 of the 128-channel atom are zeroed.
 template <int D>
-__global__ void __launch_bounds__(D < 128 ? 128 : D) k_quant_vt(QuantVtArgs a, int* status) {
-  constexpr int NT = D < 128 ? 128 : D;
+__global__ void __launch_bounds__(128) k_quant_vt(QuantVtArgs a, int* status) {
   constexpr int NAV = (D + 127) / 128;
-  constexpr int LD = D + 8;   // padded row (bf16 elements) of the staging tile
-  __shared__ __align__(16) __nv_bfloat16 tile[64 * LD];
-  const int nch = a.N / 64;
-  const int bh = blockIdx.x / nch, ch = blockIdx.x % nch;
-  const int b = bh / a.H, h = bh % a.H;
-  const __nv_bfloat16* src = a.v + b * a.sb + h * a.sh + (long long)ch * 64 * a.sn;
+  constexpr int LD = D + 8;                     // padded staging row (bf16 elements)
+  constexpr int LOADS = 32 * (D / 8) / 128;     // 16-byte loads per thread
+  __shared__ __align__(16) __nv_bfloat16 tile[32 * LD];
+  __shared__ float rtab[256];
+  fill_recip_table(rtab, threadIdx.x, 128);
+  const int n32 = a.N / 32;
   bool bad = false;
-  for (int it = threadIdx.x; it < 64 * (D / 8); it += NT) {
-    const int t = it / (D / 8), part = it % (D / 8);
-    const uint4 raw = *reinterpret_cast<const uint4*>(src + t * a.sn + part * 8);
-    *reinterpret_cast<uint4*>(&tile[t * LD + part * 8]) = raw;
-  }
-  __syncthreads();
-  const int c = threadIdx.x;
-  if (c < D) {
-    uint32_t w[8];
-    uint32_t word = 0;
+  for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
+    const int bh = u / n32, t32 = u % n32;
+    const int ch = t32 >> 1, hb = t32 & 1;
+    const int b = bh / a.H, h = bh % a.H;
+    const __nv_bfloat16* src = a.v + b * a.sb + h * a.sh + (long long)t32 * 32 * a.sn;
+    uint4 raw[LOADS];
 #pragma unroll
-    for (int blk = 0; blk < 4; ++blk) {
-      float x[16];
-      float amax = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        x[e] = __bfloat162float(tile[(blk * 16 + e) * LD + c]);
-        bad |= !isfinite(x[e]);
-        amax = fmaxf(amax, fabsf(x[e]));
-      }
-      float R;
-      const uint32_t sc = block_scale(amax, R);
-      float lo[8], hi[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) { lo[e] = x[e]; hi[e] = x[8 + e]; }
-      w[2 * blk] = encode8(lo, R);
-      w[2 * blk + 1] = encode8(hi, R);
-      word |= sc << (8 * blk);
+    for (int k = 0; k < LOADS; ++k) {
+      const int it = threadIdx.x + k * 128;
+      raw[k] = *reinterpret_cast<const uint4*>(src + (it / (D / 8)) * a.sn + (it % (D / 8)) * 8);
     }
-    uint4* dst = reinterpret_cast<uint4*>(a.codes + ((long long)bh * D + c) * (a.N / 2) + ch * 32);
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    uint8_t* atom = a.sf + (((long long)bh * nch + ch) * NAV + c / 128) * 512;
-    *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(c % 128, 0)) = word;
-  } else if (c < 128) {
-    uint8_t* atom = a.sf + ((long long)bh * nch + ch) * NAV * 512;
-    *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(c, 0)) = 0u;
+    __syncthreads();                            // previous unit's readers are done with the tile
+#pragma unroll
+    for (int k = 0; k < LOADS; ++k) {
+      const int it = threadIdx.x + k * 128;
+      *reinterpret_cast<uint4*>(&tile[(it / (D / 8)) * LD + (it % (D / 8)) * 8]) = raw[k];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = threadIdx.x; c < D; c += 128) {
+      uint32_t w[4];
+      uint32_t sc2 = 0;
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        float2 x[8];
+        float amax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[e] = make_float2(__bfloat162float(tile[(blk * 16 + 2 * e) * LD + c]),
+                             __bfloat162float(tile[(blk * 16 + 2 * e + 1) * LD + c]));
+          amax = max3_abs_nan(amax, x[e].x, x[e].y);
+        }
+        bad |= !isfinite(amax);
+        float R;
+        sc2 |= block_scale_tab(amax, rtab, R) << (8 * blk);
+        const float2 R2 = make_float2(R, R);
+        float2 lo[4], hi[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          lo[e] = __fmul2_rn(x[e], R2);
+          hi[e] = __fmul2_rn(x[4 + e], R2);
+        }
+        w[2 * blk] = encode8_pairs(lo);
+        w[2 * blk + 1] = encode8_pairs(hi);
+      }
+      *reinterpret_cast<uint4*>(a.codes + ((long long)bh * D + c) * (a.N / 2) + ch * 32 + hb * 16) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+      uint8_t* atom = a.sf + (((long long)bh * (a.N / 64) + ch) * NAV + c / 128) * 512;
+      *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(c % 128, 2 * hb)) = (uint16_t)sc2;
+    }
+    if (D < 128) {
+      for (int it = threadIdx.x; it < 128 - D; it += 128) {
+        uint8_t* atom = a.sf + ((long long)bh * (a.N / 64) + ch) * NAV * 512;
+        *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(D + it, 2 * hb)) = 0;
+      }
+    }
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }

@@ -19,7 +19,7 @@
  *     elements (NVFP4-style), no second-level scale.  scale = E4M3_RN(amax * RN(1/6)),
  *     R = RN(1/scale) (R = 0 when scale == 0), code = E2M1_RN_satfinite(x * R).
  *   - exp2 in the softmax: the method's own deterministic approximation E(x) (clamp to
- *     -127, floor split, cubic Horner in fp32 fma, exponent insert); see own_exp2().
+ *     -127, floor split, quadratic Horner in fp32 fma, exponent insert); see own_exp2().
  *   - m_new = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e)/sqrt(d)),
  *     P = E(RN(fma(S, c, -m_new))), alpha = E(RN(m_old - m_new)),
  *     a block's scale comes from E(fma(blockmax(S), c, -m_new)) (equal to the block amax
@@ -125,17 +125,17 @@ static uint8_t e4m3_encode_pos(float x) {
 
 /* ------------------------------------------------------------------ own exp2 E(x) */
 
-/* Coefficients of p(f) = 1 + c1 f + c2 f^2 + c3 f^3 ~ 2^f on [0,1): a minimax fit of the
- * relative error with p(0) = 1 held exact (max relative error 8.6e-5), rounded to fp32. */
-#define EXP2_C1 0x1.63e65ap-1f
-#define EXP2_C2 0x1.d23788p-3f
-#define EXP2_C3 0x1.3baaa8p-4f
+/* Coefficients of p(f) = 1 + c1 f + c2 f^2 ~ 2^f on [0,1): a minimax fit of the relative
+ * error with p(0) = 1 held exact (max relative error 2.05e-3, far below the spacing of the
+ * 4-bit codes P is rounded to), rounded to fp32. */
+#define EXP2_C1 0x1.54f8d6p-1f
+#define EXP2_C2 0x1.51d9ccp-2f
 
 static float own_exp2(float x) {
     float xc = fmaxf(x, -127.0f);            /* fmaxf(NaN,-127) = -127; -inf -> -127 */
     float n = floorf(xc);
     float f = xc - n;                        /* exact */
-    float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);
+    float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);
     uint32_t bits = f32_bits(p) + ((uint32_t)(int32_t)n << 23);
     return bits_f32(bits);                   /* p * 2^n; exactly 0 for xc = -127 */
 }

@@ -1,6 +1,6 @@
 """Pins of the method's own exp2 approximation E(x) used for the softmax weights.
 
-E(x) = p(f) * 2^n with n = floor(max(x, -127)), f = x - n and p a cubic with p(0) = 1;
+E(x) = p(f) * 2^n with n = floor(max(x, -127)), f = x - n and p a quadratic with p(0) = 1;
 its properties are pinned against numpy's exp2 (a library routine) and closed forms.
 """
 import numpy as np
@@ -15,14 +15,14 @@ def test_relative_error_bound_exhaustive_one_octave(orc):
     x = _all_f32_in(0xBF800000, 0xC0000000)
     e = orc.exp2(x).astype(np.float64)
     rel = np.abs(e / np.exp2(x.astype(np.float64)) - 1)
-    assert rel.max() <= 9e-5
+    assert rel.max() <= 2.1e-3
 
 
 def test_relative_error_bound_sampled_range(orc):
     rng = np.random.default_rng(3)
     x = rng.uniform(-126, 0.5, 2_000_000).astype(np.float32)
     e = orc.exp2(x).astype(np.float64)
-    assert np.max(np.abs(e / np.exp2(x.astype(np.float64)) - 1)) <= 9e-5
+    assert np.max(np.abs(e / np.exp2(x.astype(np.float64)) - 1)) <= 2.1e-3
 
 
 def test_integers_exact_and_underflow(orc):
