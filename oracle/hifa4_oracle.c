@@ -22,8 +22,9 @@
  *     -127, floor split, quadratic Horner in fp32 fma, exponent insert); see own_exp2().
  *   - m_new = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e)/sqrt(d)),
  *     P = E(RN(fma(S, c, -m_new))), alpha = E(RN(m_old - m_new)),
- *     a block's scale comes from E(fma(blockmax(S), c, -m_new)) (equal to the block amax
- *     of P because E is monotone -- pinned by a test),
+ *     a block's scale sigma comes from E(fma(blockmax(S), c, -m_new)) (equal to the block
+ *     amax of P because E is monotone -- pinned by a test), and a score's P_hat code is
+ *     the E2M1 rounding of P/sigma evaluated in the log domain (phat_value()),
  *     l = fp16_RN(fma(alpha, l, r)), r = exact sum of the tile's P_hat,
  *     O = alpha*O (fp32) + (exact tile P_hat V_hat rounded to fp32),
  *     out = bf16_RN(RN(O / l)).
@@ -138,6 +139,33 @@ static float own_exp2(float x) {
     float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);
     uint32_t bits = f32_bits(p) + ((uint32_t)(int32_t)n << 23);
     return bits_f32(bits);                   /* p * 2^n; exactly 0 for xc = -127 */
+}
+
+/* ------------------------------------------------------------------ P_hat codes */
+
+/* L(sigma) = RN_fp32(-log2(sigma)) of a positive E4M3 scale, from its integer parts:
+ * normal sigma = (8 + m) * 2^(e - 10) gives (10 - e) - log2(8 + m); subnormal
+ * sigma = m * 2^-9 gives 9 - log2(m); each computed in double, rounded once to fp32. */
+static float neg_log2_scale(uint8_t code) {
+    int e = (code >> 3) & 15, m = code & 7;
+    double v = (e == 0) ? 9.0 - log2((double)m) : (double)(10 - e) - log2((double)(8 + m));
+    return (float)v;
+}
+
+/* The value whose E2M1 rounding is the P_hat code of a score: P / sigma evaluated in the
+ * log domain.  Per block, B = RN(RN(L(sigma) - m) + 125) / 128; per score,
+ * u = min(1, max(0, RN(S * (c/128) + B)))   (NaN -> 0), k = floor(128 u), f = 128 u - k,
+ * y = p(f) * 2^(k - 125) with the exp2 polynomial p, i.e. y ~ 2^(S c - m) / sigma with the
+ * exponent argument held in [-125, 3] (outside it every code is already 0 or saturated). */
+static float phat_value(float S, float c, float B) {
+    float u = fmaf(S, c * 0.0078125f, B);
+    if (!(u > 0.0f)) u = 0.0f;
+    if (u > 1.0f) u = 1.0f;
+    float x = u * 128.0f;                 /* exact */
+    float k = floorf(x);
+    float f = x - k;                      /* exact */
+    float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);
+    return ldexpf(p, (int)k - 125);       /* exact: p in [1,2), result normal */
 }
 
 /* ------------------------------------------------------------------ block quantiser */
@@ -421,11 +449,12 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
                 float amax = own_exp2(fmaf(bmax, c, -mref));  /* = block amax of P (E monotone) */
                 uint8_t sc = e4m3_encode_pos(amax * (1.0f / 6.0f));
                 float sigma = e4m3_value(sc);
-                float R = (sigma == 0.0f) ? 0.0f : 1.0f / sigma;
+                float B = -INFINITY;                          /* sigma == 0: every code is 0 */
+                if (sigma > 0.0f) B = ((neg_log2_scale(sc) - mref) + 125.0f) * 0.0078125f;
                 for (int e = 0; e < 16; ++e) {
                     int kk = blk * 16 + e;
                     float p = own_exp2(fmaf(Sf[kk], c, -mref));
-                    uint8_t code = e2m1_encode(p * R);
+                    uint8_t code = e2m1_encode(phat_value(Sf[kk], c, B));
                     P[kk] = p;
                     Ph[kk] = (double)e2m1_value(code) * sigma;
                 }
@@ -592,6 +621,12 @@ OR_EXPORT int or_attn_bruteforce(const uint16_t* q, const uint16_t* k, const uin
 }
 
 OR_EXPORT uint16_t or_f16_bits(float f) { return f16_bits(f); }
+
+OR_EXPORT float or_neg_log2_scale(uint8_t code) { return neg_log2_scale(code); }
+
+OR_EXPORT void or_phat_values(const float* S, size_t n, float c, float B, float* y) {
+    for (size_t i = 0; i < n; ++i) y[i] = phat_value(S[i], c, B);
+}
 
 OR_EXPORT int or_num_threads(void) {
 #ifdef _OPENMP
