@@ -53,7 +53,7 @@ struct AttnCfg {
   static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
   static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
-  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 256 x fp32 reciprocal table
+  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 128 x fp32 table of L(sigma)
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
   static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 128 * 4;
   // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
@@ -93,6 +93,7 @@ struct AttnParams {
   float c;                  // RN(log2(e) / sqrt(D))
   unsigned long long wait_ns;
   int inject;               // 1: the producer never delivers kv tile 1 (timeout test)
+  float lneg[128];          // L(sigma) = RN(-log2 sigma) per E4M3 scale code (-inf for 0)
 };
 
 // Keep the register results of tcgen05.ld from being read before tcgen05.wait::ld.
@@ -182,7 +183,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     for (int i = t; i < (int)C::SZ_ONES / 4; i += nt2) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
     for (int i = t; i < 128; i += nt2) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
     fence_proxy_async_smem();
-    fill_recip_table(rtab, t, nt2);
+    for (int i = t; i < 128; i += nt2) rtab[i] = p.lneg[i];
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -387,22 +388,22 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         pmax[bl] = e2.x;
         pmax[bl + 1] = e2.y;
       }
+      const float c7 = c * 0.0078125f;
       uint32_t words[CW / 8];
       uint32_t sfw = 0;
 #pragma unroll
       for (int bl = 0; bl < NB; ++bl) {
-        float R;
-        const uint32_t sc = block_scale_tab(pmax[bl], rtab, R);
+        const uint32_t sc = cvt_e4m3(__fmul_rn(pmax[bl], kSixth));
         sfw |= sc << (8 * bl);
-        const float2 R2 = make_float2(R, R);
+        // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
+        const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
           float2 y[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int e = bl * 16 + h8 * 8 + 2 * k;
-            const float2 t2 = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2);
-            y[k] = __fmul2_rn(exp2_own2(t2), R2);
+            y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
           }
           words[2 * bl + h8] = encode8_pairs(y);
         }

@@ -119,6 +119,22 @@ bool set_smem(K kernel, uint32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
+// L(sigma) = RN_fp32(-log2 sigma) for every non-negative E4M3 scale code, from integer
+// logs in double: normal sigma = (8 + m) 2^(e - 10) gives (10 - e) - log2(8 + m),
+// subnormal sigma = m 2^-9 gives 9 - log2(m); code 0 (sigma = 0) and the NaN code map to
+// -inf.
+void fill_neg_log2_scales(float* t) {
+  for (int code = 0; code < 128; ++code) {
+    const int e = (code >> 3) & 15, m = code & 7;
+    if (code == 0 || code == 0x7F) {
+      t[code] = -INFINITY;
+      continue;
+    }
+    const double v = (e == 0) ? 9.0 - std::log2((double)m) : (double)(10 - e) - std::log2((double)(8 + m));
+    t[code] = (float)v;
+  }
+}
+
 template <int D, int BC>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                 int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
@@ -149,6 +165,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   p.c = (float)(1.4426950408889634074 / std::sqrt((double)D));
   p.wait_ns = g_wait_ns;
   p.inject = g_inject;
+  fill_neg_log2_scales(p.lneg);
   const unsigned grid = (unsigned)(B * Hq * (N / 128));
   k_attn_fwd<D, BC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
