@@ -45,13 +45,13 @@ class Workload:
 WORKLOADS = {
     "tiny": Workload("tiny", 0, 1, 1, 1, 256, 64, False, 0.5, 64,
                      None, 4, 8.0, True),
-    "qwen3-8b-4k": Workload("qwen3-8b-4k", 1, 1, 32, 8, 4096, 128, True, 0.5, 128,
+    "qwen3-8b-4k": Workload("qwen3-8b-4k", 1, 1, 32, 8, 4096, 128, True, 0.5, 256,
                             1e6, 8, 10.0, True),
     "gemma2-9b-8k": Workload("gemma2-9b-8k", 2, 1, 16, 8, 8192, 256, True, 0.25, 64,
                              1e4, 8, 4.0, True),
-    "llama3.1-8b-b4-16k": Workload("llama3.1-8b-b4-16k", 3, 4, 32, 8, 16384, 128, True, None, 128,
+    "llama3.1-8b-b4-16k": Workload("llama3.1-8b-b4-16k", 3, 4, 32, 8, 16384, 128, True, None, 256,
                                    5e5, 8, 10.0, False),
-    "phi-32k": Workload("phi-32k", 4, 1, 24, 8, 32768, 128, True, 0.5, 128,
+    "phi-32k": Workload("phi-32k", 4, 1, 24, 8, 32768, 128, True, 0.5, 256,
                         1e4, 6, 6.0, False),
 }
 

@@ -36,13 +36,14 @@ struct AttnCfg {
   static constexpr int D = D_, BC = BC_, BR = 128;
   static constexpr int KQ = D / 64;             // 64-wide K chunks of QK^T
   static constexpr int KP = BC / 64;            // 64-wide K chunks of PV
+  static constexpr int NAK = BC > 128 ? BC / 128 : 1;   // 128-row scale atoms per K tile
   static constexpr int NAV = (D + 127) / 128;   // 128-channel scale atoms of V^T
   static constexpr int QROW = D / 2, PROW = BC / 2;
   static constexpr int KS = 3, VS = 3;
   static constexpr uint32_t LQ = layout_code(QROW), LP = layout_code(PROW);
   static constexpr uint32_t SZ_Q = BR * QROW, SZ_K = BC * QROW, SZ_V = D * PROW, SZ_P = BR * PROW;
   static constexpr uint32_t SZ_ONES = 16 * PROW;
-  static constexpr uint32_t SZ_QSF = KQ * 512, SZ_KSF = KQ * 512, SZ_VSF = KP * NAV * 512, SZ_PSF = KP * 512;
+  static constexpr uint32_t SZ_QSF = KQ * 512, SZ_KSF = NAK * KQ * 512, SZ_VSF = KP * NAV * 512, SZ_PSF = KP * 512;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + align_up(SZ_Q, 1024);
   static constexpr uint32_t OFF_V = OFF_K + KS * align_up(SZ_K, 1024);
@@ -61,14 +62,17 @@ struct AttnCfg {
   static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 6 + 2;
   static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-B alignment
-  // TMEM columns
-  static constexpr uint32_t T_S = 0, T_O = 2 * BC, T_R = T_O + D, T_SFQ = T_R + 16;
-  static constexpr uint32_t T_SFK = T_SFQ + 4 * KQ, T_SFP = T_SFK + 8 * KQ, T_SFV = T_SFP + 8 * KP;
+  // TMEM columns.  S is double-buffered when it fits; a single buffer is enough for
+  // overlap because the softmax warps release S as soon as it is in their registers.
+  static constexpr uint32_t SF_COLS = 4 * KQ + 8 * KQ * NAK + 8 * KP + 8 * KP * NAV + 4;
+  static constexpr int SB = (2 * BC + D + 16 + SF_COLS <= 512) ? 2 : 1;
+  static constexpr uint32_t T_S = 0, T_O = SB * BC, T_R = T_O + D, T_SFQ = T_R + 16;
+  static constexpr uint32_t T_SFK = T_SFQ + 4 * KQ, T_SFP = T_SFK + 8 * KQ * NAK, T_SFV = T_SFP + 8 * KP;
   static constexpr uint32_t T_SF1 = T_SFV + 8 * KP * NAV, T_END = T_SF1 + 4;
   static constexpr uint32_t TMEM_COLS = T_END <= 256 ? 256 : 512;
   static_assert(T_END <= 512, "TMEM budget exceeded");
   static_assert(D == 64 || D == 128 || D == 256, "head dim");
-  static_assert(BC == 64 || BC == 128, "kv tile");
+  static_assert(BC == 64 || BC == 128 || BC == 256, "kv tile");
   // softmax warpgroups: each takes CW consecutive score columns of every row and D/NSW
   // columns of O (both at least 32, the width of one tcgen05.ld)
 #ifndef HIFA4_MAX_NSW
@@ -164,7 +168,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   const int bh = blockIdx.x % BH;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
-  const int nt = p.causal ? ((qtile + 1) * 128) / BC : p.N / BC;
+  const int nt = p.causal ? ((qtile + 1) * 128 + BC - 1) / BC : p.N / BC;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
@@ -211,7 +215,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         mbar_arrive_expect_tx(&k_full[ks], C::SZ_K + C::SZ_KSF);
         tma_load_2d(sK(ks), &tmK, 0, kvh * p.N + j * BC, &k_full[ks]);
         const int katom = (j * BC) / 128;
-        bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * C::SZ_KSF, C::SZ_KSF, &k_full[ks]);
+        // the tile's NAK consecutive 128-row atoms (KQ x 512 bytes each) are contiguous
+        bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * (C::KQ * 512), C::SZ_KSF, &k_full[ks]);
         if (j >= C::VS && !mbar_wait(&v_empty[vs], ((j / C::VS) - 1) & 1, abort, p.status, p.wait_ns)) {
           issued = 2 * j + 1;
           break;
@@ -280,9 +285,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       __syncwarp();
     }
     for (int j = 0; ok && j < nt; ++j) {
-      const int ks = j % C::KS, sb = j & 1;
+      const int ks = j % C::KS, sb = j % C::SB;
       ok = wait_all(&k_full[ks], (j / C::KS) & 1, abort, p.status, p.wait_ns);
-      if (ok && j >= 2) ok = wait_all(&s_empty[sb], ((j >> 1) - 1) & 1, abort, p.status, p.wait_ns);
+      if (ok && j >= C::SB) ok = wait_all(&s_empty[sb], ((j / C::SB) - 1) & 1, abort, p.status, p.wait_ns);
       if (!ok) break;
       if (BC == 64 && (j & 1)) {
         // keys 64..127 of the 128-row scale atom: move record words 2,3 into words 0,1
@@ -297,15 +302,19 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       }
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t sfk = tbase + C::T_SFK + sb * 4 * C::KQ;
+        // K scale atoms (row atom rt, chunk kc) -> 4 columns at chunk kc's 4*NAK columns + 4 rt
+        const uint32_t sfk = tbase + C::T_SFK + (j & 1) * 4 * C::KQ * C::NAK;
 #pragma unroll
-        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(sfk + 4 * kc, sKsf(ks) + 512 * kc);
+        for (int rt = 0; rt < C::NAK; ++rt)
+#pragma unroll
+          for (int kc = 0; kc < C::KQ; ++kc)
+            tmem_cp_sf_atom(sfk + 4 * (C::NAK * kc + rt), sKsf(ks) + 512 * (rt * C::KQ + kc));
         const uint32_t aK = smem_u32(sK(ks));
 #pragma unroll
         for (int kc = 0; kc < C::KQ; ++kc)
           mma_nvf4(tbase + C::T_S + sb * BC, smem_desc(aQ + 32 * kc, 0, 8 * C::QROW, C::LQ),
-                   smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc, sfk + 4 * kc,
-                   kc > 0 ? 1u : 0u);
+                   smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc,
+                   sfk + 4 * C::NAK * kc, kc > 0 ? 1u : 0u);
         tc_commit(&s_full[sb]);
         tc_commit(&k_empty[ks]);
       }
@@ -334,8 +343,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      const int sb = j & 1;
-      ok = wait_all(&s_full[sb], (j >> 1) & 1, abort, p.status, p.wait_ns);
+      const int sb = j % C::SB, pb = j & 1;
+      ok = wait_all(&s_full[sb], (j / C::SB) & 1, abort, p.status, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       float s[CW];
@@ -408,13 +417,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           words[2 * bl + h8] = encode8_pairs(y);
         }
       }
-      uint8_t* pbuf = sP(sb);
+      uint8_t* pbuf = sP(pb);
 #pragma unroll
       for (int q = 0; q < CW / 32; ++q)
         *reinterpret_cast<uint4*>(pbuf + swz_offset(row, col0 / 32 + q, C::PROW)) =
             make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
       {
-        uint8_t* atom = sPsf(sb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
+        uint8_t* atom = sPsf(pb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
         if (NB == 4) *reinterpret_cast<uint32_t*>(atom) = sfw;
         else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
       }
@@ -448,7 +457,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[sb]);
+      if (lane == 0) mbar_arrive(&p_full[pb]);
       alpha_prev = alpha;
       m_run = mnew;
     }

@@ -285,9 +285,11 @@ int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, con
   if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : 128;
-  if (kv_tile != 64 && kv_tile != 128) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : (d == 128 ? 256 : 128);
+  if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 64 && kv_tile == 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (N % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q, B, Hq, N, d, 0) || !qt_ok(k, B, Hkv, N, d, 0) || !qt_ok(vt, B, Hkv, N, d, 1))
     return HIFA4_ERR_INVALID_ARG;
   if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
@@ -296,6 +298,7 @@ int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, con
     return kv_tile == 64 ? launch_attn<64, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
                          : launch_attn<64, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
   } else if (d == 128) {
+    if (kv_tile == 256) return launch_attn<128, 256>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
     return kv_tile == 64 ? launch_attn<128, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
                          : launch_attn<128, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
   }

@@ -135,13 +135,17 @@ HIFA4_API int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B,
  *   S      = Q_hat K_hat_j^T                     (4-bit tensor-core MMA, fp32 accumulate)
  *   m_new  = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e) / sqrt(d))
  *   P      = E(RN(fma(S, c, -m_new)))            (E: the library's deterministic exp2)
- *   P_hat  = 4-bit blocks of 16 keys, each block's scale from E(fma(blockmax S, c, -m_new))
+ *   P_hat  = 4-bit blocks of 16 keys, each block's scale sigma from E(fma(blockmax S, c,
+ *            -m_new)); a score's code is the E2M1 rounding of y = p(frac(128u)) *
+ *            2^(floor(128u) - 125), u = sat(S c/128 + (RN(-log2 sigma) - m_new + 125)/128),
+ *            i.e. of P / sigma evaluated in the log domain
  *   alpha  = E(m - m_new)  (0 on the first tile)
  *   O      = alpha * O + P_hat V_hat_j           (4-bit MMA)
  *   r      = P_hat * 1                           (4-bit MMA against ones: P-Reordering)
  *   l      = fp16_RN(fma(alpha, l, r)),  m = m_new
- * and finally out = bf16_RN(O / l).  kv_tile is 64 or 128 (0 selects 128 for d <= 128 and
- * 64 for d = 256; d = 256 supports only 64) and is part of the result's definition.
+ * and finally out = bf16_RN(O / l).  kv_tile is 64, 128 or 256 and is part of the result's
+ * definition; N must be a multiple of it.  0 selects 128 for d = 64, 256 for d = 128 and
+ * 64 for d = 256; d = 256 supports only 64 and d = 64 at most 128.
  * o: bf16 [B, Hq, N, d] dense.  m_out, l_out: fp16 [B, Hq, N] dense, or NULL.
  */
 HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,

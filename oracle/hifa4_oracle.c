@@ -397,9 +397,9 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
         for (int x = 0; x < d; ++x) qd[x] = bf16_to_f32(a->q[row * d + x]);
 
     for (int j = 0; j < ntiles; ++j) {
-        double S[128];
-        float Sf[128];
-        int valid[128];
+        double S[256];
+        float Sf[256];
+        int valid[256];
         double rowmax = -INFINITY;
         for (int kk = 0; kk < bc; ++kk) {
             int key = j * bc + kk;
@@ -440,7 +440,7 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
         }
 
         /* P and P_hat of the tile */
-        double P[128], Ph[128];
+        double P[256], Ph[256];
         for (int kk = 0; kk < bc; ++kk) { P[kk] = 0.0; Ph[kk] = 0.0; }
         if (a->quant) {
             for (int blk = 0; blk < bc / 16; ++blk) {
@@ -541,7 +541,7 @@ OR_EXPORT int or_attn_fwd(const uint8_t* qc, const uint8_t* qs, const uint8_t* k
                           int causal, int bc, int state, int l_from_p, int s_model,
                           const long long* rows, long long nrows,
                           double* o_f64, uint16_t* o_bf16, float* m_out, float* l_out) {
-    if (d % 16 || d > 256 || bc % 16 || bc > 128 || N % bc || Hq % Hkv) return -1;
+    if (d % 16 || d > 256 || bc % 16 || bc > 256 || N % bc || Hq % Hkv) return -1;
     loop_args a = {qc, qs, kc, ks, vtc, vts, NULL, NULL, NULL, B, Hq, Hkv, N, d, causal, bc,
                    1, state, l_from_p, s_model};
     long long n = rows ? nrows : (long long)B * Hq * N;
@@ -560,7 +560,7 @@ OR_EXPORT int or_attn_fwd(const uint8_t* qc, const uint8_t* qs, const uint8_t* k
 OR_EXPORT int or_attn_loop_exact(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
                                  int Hkv, int N, int d, int causal, int bc,
                                  const long long* rows, long long nrows, double* o_f64) {
-    if (d > 256 || bc > 128 || N % bc || Hq % Hkv) return -1;
+    if (d > 256 || bc > 256 || N % bc || Hq % Hkv) return -1;
     loop_args a = {NULL, NULL, NULL, NULL, NULL, NULL, q, k, v, B, Hq, Hkv, N, d, causal, bc,
                    0, ST_F64, 0, 0};
     long long n = rows ? nrows : (long long)B * Hq * N;
@@ -577,7 +577,7 @@ OR_EXPORT int or_attn_trace(const uint8_t* qc, const uint8_t* qs, const uint8_t*
                             const uint8_t* vtc, const uint8_t* vts, int B, int Hq, int Hkv, int N, int d,
                             int causal, int bc, int state, int l_from_p, int s_model, long long row,
                             float* tr_m, float* tr_p, float* tr_phat, double* o_f64, float* ml) {
-    if (d % 16 || d > 256 || bc % 16 || bc > 128 || N % bc || Hq % Hkv) return -1;
+    if (d % 16 || d > 256 || bc % 16 || bc > 256 || N % bc || Hq % Hkv) return -1;
     loop_args a = {qc, qs, kc, ks, vtc, vts, NULL, NULL, NULL, B, Hq, Hkv, N, d, causal, bc,
                    1, state, l_from_p, s_model};
     row_out o = {o_f64, NULL, 0, 0, tr_m, tr_p, tr_phat};

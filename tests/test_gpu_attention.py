@@ -14,7 +14,9 @@ REDUCED = [
     ("tiny", {}),
     ("tiny", dict(causal=True)),
     ("qwen3-8b-4k", dict(Hq=4, Hkv=2, N=512)),
-    ("qwen3-8b-4k", dict(Hq=4, Hkv=2, N=384, causal=False)),
+    ("qwen3-8b-4k", dict(Hq=4, Hkv=2, N=512, bc=128)),
+    ("qwen3-8b-4k", dict(Hq=4, Hkv=2, N=384, bc=128, causal=False)),
+    ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=768, causal=False)),
     ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=256, bc=64)),
     ("gemma2-9b-8k", dict(Hq=4, Hkv=2, N=512)),
     ("gemma2-9b-8k", dict(Hq=2, Hkv=1, N=256, causal=False)),
