@@ -1,9 +1,9 @@
 """Benchmark of the HiFA4-style 4-bit attention forward on B200.
 
 One step = the whole hot path over one batch of the Qwen3-8B-shaped 4k causal workload
-(B=1, Hq=32, Hkv=8, N=4096, d=128): Smooth-QK + 4-bit quantisation of Q and K, 4-bit
-quantisation of V^T, and the fused 4-bit attention kernel, each launched through the C
-ABI (libhifa4.so).  Metric: TFLOPS = 4*B*Hq*N^2*d / 2 (causal) per step / step time.
+(B=1, Hq=32, Hkv=8, N=4096, d=128): Smooth-QK + 4-bit quantisation of Q and K and 4-bit
+quantisation of V^T (one launch, hifa4_quantize_qkv), then the fused 4-bit attention
+kernel (hifa4_attn_fwd_quantized), both through the C ABI (libhifa4.so).  Metric: TFLOPS = 4*B*Hq*N^2*d / 2 (causal) per step / step time.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -163,15 +163,12 @@ def run_gpu(args):
         j = i & 1
         if ev is not None:
             ev[0].record(stream)
-        hifa4.hifa4_quantize_qk(qt, kt, s, sinv, status=st, out=(qq[j], kq[j]))
+        hifa4.hifa4_quantize_qkv(qt, kt, vt, s, sinv, status=st, out=(qq[j], kq[j], vq[j]))
         if ev is not None:
             ev[1].record(stream)
-        hifa4.hifa4_quantize_v(vt, status=st, out=vq[j])
-        if ev is not None:
-            ev[2].record(stream)
         hifa4.hifa4_attn_fwd_quantized(qq[j], kq[j], vq[j], causal=w.causal, kv_tile=w.bc, status=st, o=o, m=m, l=l)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     for i in range(args.warmup):
         step(i)
@@ -180,7 +177,7 @@ def run_gpu(args):
         raise RuntimeError(f"warm-up reported {hifa4.status_string(code)}")
 
     # timed region: K steps, barrier + synchronize on both sides, per-kernel events inside
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     if dist is not None:
@@ -200,9 +197,8 @@ def run_gpu(args):
     code = hifa4.hifa4_read_status(st)
     if code != hifa4.OK:
         raise RuntimeError(f"timed steps reported {hifa4.status_string(code)}")
-    k_qk = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    k_v = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    k_attn = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    k_quant = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    k_attn = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
 
     # e2e through the public API with host buffers: H2D of Q, K, V from pinned memory,
     # the hot path, D2H of O, m, l -- every step
@@ -232,8 +228,7 @@ def run_gpu(args):
     elapsed = reduce_max(elapsed, dist, device)
     e2e_ms = reduce_max(e2e_ms, dist, device)
     k_attn = reduce_max(k_attn, dist, device)
-    k_qk = reduce_max(k_qk, dist, device)
-    k_v = reduce_max(k_v, dist, device)
+    k_quant = reduce_max(k_quant, dist, device)
     agg = aggregate([elapsed] * world, flops, args.steps)
     e2e = aggregate([e2e_ms] * world, flops, e2e_steps)
     h2d = sum(x.numel() * x.element_size() for x in host)
@@ -242,7 +237,7 @@ def run_gpu(args):
     hbm, bf16, src = peaks()
     fp4_peak = bf16 * FP4_OVER_BF16
     achieved = flops / (k_attn * 1e-3) / 1e12
-    qk_bytes = (B * (Hq + Hkv) * N * d) * (2 + 0.5 + 1 / 16)
+    quant_bytes = (B * (Hq + 2 * Hkv) * N * d) * (2 + 0.5 + 1 / 16)
     out = {
         "metric": "4-bit attn fwd TFLOPS (4*B*Hq*N^2*d, causal/2) and % of B200 dense FP4 peak",
         "value": round(agg["tflops"], 3),
@@ -262,16 +257,16 @@ def run_gpu(args):
         "pct_fp4_peak": round(100 * agg["tflops"] / world / fp4_peak, 2),
         "pct_fp4_peak_datasheet_9pf": round(100 * agg["tflops"] / world / 9000.0, 2),
         "tokens_per_s": round(B * N * world / (agg["ms_per_step"] * 1e-3), 1),
-        "kernels_us": {"quantize_qk": round(k_qk * 1e3, 2), "quantize_v": round(k_v * 1e3, 2),
-                       "attn_fwd": round(k_attn * 1e3, 2)},
+        "kernels_us": {"quantize_qkv": round(k_quant * 1e3, 2), "attn_fwd": round(k_attn * 1e3, 2)},
         "attn_kernel_tflops": round(achieved, 2),
-        "quantize_qk_gbs": round(qk_bytes / (k_qk * 1e-3) / 1e9, 1),
+        "quantize_qkv_gbs": round(quant_bytes / (k_quant * 1e-3) / 1e9, 1),
+        "quantize_qkv_frac_hbm": round(quant_bytes / (k_quant * 1e-3) / 1e9 / hbm, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": None,
                      "peak_source": f"{src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)"},
         "e2e": {"value": round(e2e["tflops"], 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -386,7 +386,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
       float mnew = m_run;
       if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
-      const float alpha = (m_run == -INFINITY) ? 0.0f : exp2_own(__fsub_rn(m_run, mnew));
+      // alpha = E(m - m_new): 0 on the first tile, exactly E(0) = 1 when the max is unchanged
+      const float alpha = (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
       const float negm = -mnew;
       const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
       // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call

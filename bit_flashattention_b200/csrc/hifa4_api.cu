@@ -279,6 +279,33 @@ int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, 
   return cuda_status(cudaGetLastError());
 }
 
+int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_t q_strides[3],
+                       const int64_t k_strides[3], const int64_t v_strides[3], int B, int Hq, int Hkv, int N, int d,
+                       const float* s, const float* sinv, const hifa4_qtensor* q_out, const hifa4_qtensor* k_out,
+                       const hifa4_qtensor* vt_out, int* status, cudaStream_t stream) {
+  if (!strides_ok(q, q_strides) || !strides_ok(k, k_strides) || !strides_ok(v, v_strides) || !status ||
+      ((s == nullptr) != (sinv == nullptr)) || (s && (!aligned16(s) || !aligned16(sinv))))
+    return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0) || !qt_ok(vt_out, B, Hkv, N, d, 1))
+    return HIFA4_ERR_INVALID_ARG;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  const int rows = d == 256 ? 64 : 128;
+  QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
+                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
+  QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
+                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
+  QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
+                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 64)};
+  const int units = qa.units + ka.units + va.units;
+  switch (d) {
+    case 64: k_quant_qkv<64><<<resident_grid(k_quant_qkv<64>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+    case 128: k_quant_qkv<128><<<resident_grid(k_quant_qkv<128>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+    default: k_quant_qkv<256><<<resident_grid(k_quant_qkv<256>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
 int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
                              int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
                              void* l_out, int* status, cudaStream_t stream) {

@@ -28,83 +28,92 @@ __device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
   return d;
 }
 
-// Grid-stride over units of ROWS rows of one head (Q units first, then K units).  Thread
+template <int D>
+struct RowsUnit {
+  static constexpr int BPR = D / 16;                  // blocks per row
+  static constexpr int RPP = 256 / BPR;               // rows per pass
+  static constexpr int ROWS = D == 256 ? 64 : 128;    // rows per unit
+  static constexpr int PASSES = ROWS / RPP;
+};
+
+// One unit (ROWS rows of one head) of the Q/K quantiser with 256 threads.  Thread
 // (row r, block k) quantises one 16-element block: two 16-byte loads (all of a thread's
-// loads in flight before any arithmetic), the block amax with 3-input max instructions, the
-// scale from the amax and its reciprocal from a shared table, 8 code bytes stored at once.
-// The four blocks of a 64-wide chunk sit in lanes 4q..4q+3, which assemble the chunk's
-// scale word with two shuffles.
+// loads in flight before any arithmetic), the block amax with 3-input max instructions,
+// the scale from the amax and its reciprocal from a shared table, 8 code bytes stored at
+// once.  The four blocks of a 64-wide chunk sit in lanes 4q..4q+3, which assemble the
+// chunk's scale word with two shuffles.
+template <int D>
+__device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit, const float* rtab, bool& bad) {
+  using U = RowsUnit<D>;
+  const int lane = threadIdx.x & 31;
+  const int blk = threadIdx.x % U::BPR;
+  const int rsub = threadIdx.x / U::BPR;
+  const int per_head = a.N / U::ROWS;
+  const int bh = unit / per_head, n0 = (unit % per_head) * U::ROWS;
+  const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
+  const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + blk * 16;
+  uint4 raw[U::PASSES][2];
+#pragma unroll
+  for (int k = 0; k < U::PASSES; ++k) {
+    const uint4* src = reinterpret_cast<const uint4*>(base + (long long)(n0 + rsub + k * U::RPP) * a.sn);
+    raw[k][0] = src[0];
+    raw[k][1] = src[1];
+  }
+  float2 s2[8];
+  if (a.scale) {
+    const float4* sp = reinterpret_cast<const float4*>(a.scale + g * D + blk * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t = __ldg(sp + q);
+      s2[2 * q] = make_float2(t.x, t.y);
+      s2[2 * q + 1] = make_float2(t.z, t.w);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < U::PASSES; ++k) {
+    const int row = n0 + rsub + k * U::RPP;
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k][0]);
+    float2 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
+    if (a.scale) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], s2[e]);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
+    bad |= !isfinite(amax);
+    float R;
+    const uint32_t sc = block_scale_tab(amax, rtab, R);
+    const float2 R2 = make_float2(R, R);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], R2);
+    const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
+    *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
+        make_uint2(encode8_pairs(lo), encode8_pairs(hi));
+    uint32_t word = sc << (8 * (lane & 3));
+    word |= __shfl_xor_sync(0xffffffffu, word, 1);
+    word |= __shfl_xor_sync(0xffffffffu, word, 2);
+    if ((lane & 3) == 0) {
+      uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
+      *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
+    }
+  }
+}
+
+// Grid-stride over Q units then K units.
 template <int D>
 __global__ void __launch_bounds__(256) k_quant_rows(QuantRowsArgs qa, QuantRowsArgs ka, int* status) {
-  constexpr int BPR = D / 16;                  // blocks per row
-  constexpr int RPP = 256 / BPR;               // rows per pass
-  constexpr int ROWS = D == 256 ? 64 : 128;    // rows per unit
-  constexpr int PASSES = ROWS / RPP;
-  const int lane = threadIdx.x & 31;
-  const int blk = threadIdx.x % BPR;
-  const int rsub = threadIdx.x / BPR;
   __shared__ float rtab[256];
   fill_recip_table(rtab, threadIdx.x, 256);
   __syncthreads();
   bool bad = false;
   for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
-    const bool isq = u < qa.units;
-    const QuantRowsArgs& a = isq ? qa : ka;
-    const int unit = isq ? u : u - qa.units;
-    const int per_head = a.N / ROWS;
-    const int bh = unit / per_head, n0 = (unit % per_head) * ROWS;
-    const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
-    const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + blk * 16;
-    uint4 raw[PASSES][2];
-#pragma unroll
-    for (int k = 0; k < PASSES; ++k) {
-      const uint4* src = reinterpret_cast<const uint4*>(base + (long long)(n0 + rsub + k * RPP) * a.sn);
-      raw[k][0] = src[0];
-      raw[k][1] = src[1];
-    }
-    float2 s2[8];
-    if (a.scale) {
-      const float4* sp = reinterpret_cast<const float4*>(a.scale + g * D + blk * 16);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 t = __ldg(sp + q);
-        s2[2 * q] = make_float2(t.x, t.y);
-        s2[2 * q + 1] = make_float2(t.z, t.w);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < PASSES; ++k) {
-      const int row = n0 + rsub + k * RPP;
-      const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k][0]);
-      float2 v[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
-      if (a.scale) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], s2[e]);
-      }
-      float amax = 0.0f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
-      bad |= !isfinite(amax);
-      float R;
-      const uint32_t sc = block_scale_tab(amax, rtab, R);
-      const float2 R2 = make_float2(R, R);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], R2);
-      const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
-      *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
-          make_uint2(encode8_pairs(lo), encode8_pairs(hi));
-      uint32_t word = sc << (8 * (lane & 3));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      if ((lane & 3) == 0) {
-        uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
-        *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
-      }
-    }
+    if (u < qa.units) quant_rows_unit<D>(qa, u, rtab, bad);
+    else quant_rows_unit<D>(ka, u - qa.units, rtab, bad);
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, ST_NONFINITE);
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }
 
 struct QuantVtArgs {
@@ -113,80 +122,105 @@ struct QuantVtArgs {
   int H, N;
   uint8_t* codes;             // [B, Hkv, D, N/2]
   uint8_t* sf;                // [B, Hkv, N/64, ceil(D/128), 512]
-  int units;                  // B * Hkv * N / 32
+  int units;                  // B * Hkv * N / TOK for the kernel's TOK
 };
 
-// Grid-stride over (b, kv head, 32-token half of a 64-token chunk) units, 128 threads.
-// The 32 x D tile is staged in shared memory with coalesced 16-byte loads (all of a
-// thread's loads in flight first); then thread c quantises the two 16-token blocks of
-// channel c in this half, writes their 16 code bytes and its 2 bytes of the channel's
-// scale word.  For D = 64 the unused rows 64..127 of the 128-channel atom are zeroed.
-template <int D>
-__global__ void __launch_bounds__(128) k_quant_vt(QuantVtArgs a, int* status) {
+// One unit (TOK consecutive tokens of one kv head, TOK = 32 with 128 threads or 64 with
+// 256 threads) of the transposing V quantiser.  The TOK x D tile is staged in shared
+// memory with coalesced 16-byte loads (all of a thread's loads in flight first); then item
+// (channel c, 32-token half) quantises the half's two 16-token blocks of channel c and
+// writes their 16 code bytes and its 2 bytes of the channel's scale word.  For D = 64 the
+// unused rows 64..127 of the 128-channel atom are zeroed.
+template <int D, int TOK, int NT>
+__device__ __forceinline__ void quant_vt_unit(const QuantVtArgs& a, int unit, __nv_bfloat16* tile, const float* rtab,
+                                              bool& bad) {
   constexpr int NAV = (D + 127) / 128;
   constexpr int LD = D + 8;                     // padded staging row (bf16 elements)
-  constexpr int LOADS = 32 * (D / 8) / 128;     // 16-byte loads per thread
-  __shared__ __align__(16) __nv_bfloat16 tile[32 * LD];
+  constexpr int LOADS = TOK * (D / 8) / NT;     // 16-byte loads per thread
+  const int nunit = a.N / TOK;
+  const int bh = unit / nunit, t0 = (unit % nunit) * TOK;
+  const int b = bh / a.H, h = bh % a.H;
+  const __nv_bfloat16* src = a.v + b * a.sb + h * a.sh + (long long)t0 * a.sn;
+  uint4 raw[LOADS];
+#pragma unroll
+  for (int k = 0; k < LOADS; ++k) {
+    const int it = threadIdx.x + k * NT;
+    raw[k] = *reinterpret_cast<const uint4*>(src + (it / (D / 8)) * a.sn + (it % (D / 8)) * 8);
+  }
+  __syncthreads();                            // the previous unit's readers are done with the tile
+#pragma unroll
+  for (int k = 0; k < LOADS; ++k) {
+    const int it = threadIdx.x + k * NT;
+    *reinterpret_cast<uint4*>(&tile[(it / (D / 8)) * LD + (it % (D / 8)) * 8]) = raw[k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int it = threadIdx.x; it < (TOK / 32) * D; it += NT) {
+    const int c = it % D, hh = it / D;
+    const int half = t0 / 32 + hh, ch = half >> 1, hb = half & 1;
+    uint32_t w[4];
+    uint32_t sc2 = 0;
+#pragma unroll
+    for (int blk = 0; blk < 2; ++blk) {
+      float2 x[8];
+      float amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        x[e] = make_float2(__bfloat162float(tile[(hh * 32 + blk * 16 + 2 * e) * LD + c]),
+                           __bfloat162float(tile[(hh * 32 + blk * 16 + 2 * e + 1) * LD + c]));
+        amax = max3_abs_nan(amax, x[e].x, x[e].y);
+      }
+      bad |= !isfinite(amax);
+      float R;
+      sc2 |= block_scale_tab(amax, rtab, R) << (8 * blk);
+      const float2 R2 = make_float2(R, R);
+      float2 lo[4], hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        lo[e] = __fmul2_rn(x[e], R2);
+        hi[e] = __fmul2_rn(x[4 + e], R2);
+      }
+      w[2 * blk] = encode8_pairs(lo);
+      w[2 * blk + 1] = encode8_pairs(hi);
+    }
+    *reinterpret_cast<uint4*>(a.codes + ((long long)bh * D + c) * (a.N / 2) + ch * 32 + hb * 16) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+    uint8_t* atom = a.sf + (((long long)bh * (a.N / 64) + ch) * NAV + c / 128) * 512;
+    *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(c % 128, 2 * hb)) = (uint16_t)sc2;
+  }
+  if constexpr (D < 128) {
+    constexpr int PAD = 128 - D;
+    for (int it = threadIdx.x; it < (TOK / 32) * PAD; it += NT) {
+      const int half = t0 / 32 + it / PAD, r = D + it % PAD;
+      uint8_t* atom = a.sf + ((long long)bh * (a.N / 64) + (half >> 1)) * NAV * 512;
+      *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(r, 2 * (half & 1))) = 0;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) k_quant_vt(QuantVtArgs a, int* status) {
+  __shared__ __align__(16) __nv_bfloat16 tile[32 * (D + 8)];
   __shared__ float rtab[256];
   fill_recip_table(rtab, threadIdx.x, 128);
-  const int n32 = a.N / 32;
   bool bad = false;
-  for (int u = blockIdx.x; u < a.units; u += gridDim.x) {
-    const int bh = u / n32, t32 = u % n32;
-    const int ch = t32 >> 1, hb = t32 & 1;
-    const int b = bh / a.H, h = bh % a.H;
-    const __nv_bfloat16* src = a.v + b * a.sb + h * a.sh + (long long)t32 * 32 * a.sn;
-    uint4 raw[LOADS];
-#pragma unroll
-    for (int k = 0; k < LOADS; ++k) {
-      const int it = threadIdx.x + k * 128;
-      raw[k] = *reinterpret_cast<const uint4*>(src + (it / (D / 8)) * a.sn + (it % (D / 8)) * 8);
-    }
-    __syncthreads();                            // previous unit's readers are done with the tile
-#pragma unroll
-    for (int k = 0; k < LOADS; ++k) {
-      const int it = threadIdx.x + k * 128;
-      *reinterpret_cast<uint4*>(&tile[(it / (D / 8)) * LD + (it % (D / 8)) * 8]) = raw[k];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int c = threadIdx.x; c < D; c += 128) {
-      uint32_t w[4];
-      uint32_t sc2 = 0;
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-        float2 x[8];
-        float amax = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] = make_float2(__bfloat162float(tile[(blk * 16 + 2 * e) * LD + c]),
-                             __bfloat162float(tile[(blk * 16 + 2 * e + 1) * LD + c]));
-          amax = max3_abs_nan(amax, x[e].x, x[e].y);
-        }
-        bad |= !isfinite(amax);
-        float R;
-        sc2 |= block_scale_tab(amax, rtab, R) << (8 * blk);
-        const float2 R2 = make_float2(R, R);
-        float2 lo[4], hi[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          lo[e] = __fmul2_rn(x[e], R2);
-          hi[e] = __fmul2_rn(x[4 + e], R2);
-        }
-        w[2 * blk] = encode8_pairs(lo);
-        w[2 * blk + 1] = encode8_pairs(hi);
-      }
-      *reinterpret_cast<uint4*>(a.codes + ((long long)bh * D + c) * (a.N / 2) + ch * 32 + hb * 16) =
-          make_uint4(w[0], w[1], w[2], w[3]);
-      uint8_t* atom = a.sf + (((long long)bh * (a.N / 64) + ch) * NAV + c / 128) * 512;
-      *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(c % 128, 2 * hb)) = (uint16_t)sc2;
-    }
-    if (D < 128) {
-      for (int it = threadIdx.x; it < 128 - D; it += 128) {
-        uint8_t* atom = a.sf + ((long long)bh * (a.N / 64) + ch) * NAV * 512;
-        *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(D + it, 2 * hb)) = 0;
-      }
-    }
+  for (int u = blockIdx.x; u < a.units; u += gridDim.x) quant_vt_unit<D, 32, 128>(a, u, tile, rtab, bad);
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+}
+
+// Q, K and V in one launch: grid-stride over Q and K row units, then 64-token V units.
+template <int D>
+__global__ void __launch_bounds__(256) k_quant_qkv(QuantRowsArgs qa, QuantRowsArgs ka, QuantVtArgs va, int* status) {
+  __shared__ __align__(16) __nv_bfloat16 tile[64 * (D + 8)];
+  __shared__ float rtab[256];
+  fill_recip_table(rtab, threadIdx.x, 256);
+  __syncthreads();
+  bool bad = false;
+  const int nrows = qa.units + ka.units;
+  for (int u = blockIdx.x; u < nrows + va.units; u += gridDim.x) {
+    if (u < qa.units) quant_rows_unit<D>(qa, u, rtab, bad);
+    else if (u < nrows) quant_rows_unit<D>(ka, u - qa.units, rtab, bad);
+    else quant_vt_unit<D, 64, 256>(va, u - nrows, tile, rtab, bad);
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }

@@ -49,6 +49,7 @@ def lib():
             "hifa4_calibrate_smooth": ([P, P, P, P, i, i, i, i, i, f, P, P, P, P], i),
             "hifa4_quantize_qk": ([P, P, P, P, i, i, i, i, i, P, P, QP, QP, P, P], i),
             "hifa4_quantize_v": ([P, P, i, i, i, i, QP, P, P], i),
+            "hifa4_quantize_qkv": ([P, P, P, P, P, P, i, i, i, i, i, P, P, QP, QP, QP, P, P], i),
             "hifa4_attn_fwd_quantized": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
             "hifa4_attn_workspace_bytes": ([i, i, i, i], sz),
             "hifa4_attn_fwd": ([QP, QP, P, P, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
@@ -151,6 +152,19 @@ def hifa4_quantize_qk(q, k, s=None, sinv=None, status=None, out=None):
     st = status if status is not None else new_status(q.device)
     _check(lib().hifa4_quantize_qk(_ptr(q), _ptr(k), _strides(q), _strides(k), B, Hq, Hkv, N, d, _ptr(s), _ptr(sinv),
                                    out[0].c(), out[1].c(), _ptr(st), _stream()), "hifa4_quantize_qk")
+    return out
+
+
+def hifa4_quantize_qkv(q, k, v, s=None, sinv=None, status=None, out=None):
+    """Smooth-QK + 4-bit Q, K and V^T in one launch -> (QTensor, QTensor, QTensor)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device), QTensor(B, Hkv, N, d, 1, q.device))
+    st = status if status is not None else new_status(q.device)
+    _check(lib().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _strides(q), _strides(k), _strides(v), B, Hq, Hkv, N, d,
+                                    _ptr(s), _ptr(sinv), out[0].c(), out[1].c(), out[2].c(), _ptr(st), _stream()),
+           "hifa4_quantize_qkv")
     return out
 
 

@@ -129,6 +129,16 @@ HIFA4_API int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B,
                      const hifa4_qtensor* vt_out, int* status, cudaStream_t stream);
 
 /*
+ * hifa4_quantize_qk and hifa4_quantize_v in one launch (same arguments and outputs; the
+ * three quantisations are independent, so V's latency hides behind Q and K).
+ */
+HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_t q_strides[3],
+                                 const int64_t k_strides[3], const int64_t v_strides[3], int B, int Hq, int Hkv,
+                                 int N, int d, const float* s, const float* sinv, const hifa4_qtensor* q_out,
+                                 const hifa4_qtensor* k_out, const hifa4_qtensor* vt_out, int* status,
+                                 cudaStream_t stream);
+
+/*
  * The fused 4-bit attention forward on already quantised Q, K and V^T.
  * For every (b, h, query row i), kv tiles j = 0, 1, ... of kv_tile keys (only tiles
  * holding a visible key when causal):

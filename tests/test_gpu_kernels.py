@@ -47,6 +47,26 @@ def test_quantisers_bit_exact(name, kw):
     assert all(res.values()), res
 
 
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", {}),
+    ("qwen3-8b-4k", dict(Hq=8, Hkv=2, N=512)),
+    ("gemma2-9b-8k", dict(Hq=4, Hkv=2, N=256)),
+    ("llama3.1-8b-b4-16k", dict(B=2, Hq=4, Hkv=2, N=256)),
+])
+def test_quantize_qkv_one_launch_bit_exact(name, kw):
+    w = configs.scaled(configs.get(name), **kw)
+    q, k, v = gen.inputs(w)
+    s, sinv = gc.smooth_scales(w)
+    st = hifa4.new_status("cuda")
+    qq, kq, vq = hifa4.hifa4_quantize_qkv(gc.bf16_dev(q), gc.bf16_dev(k), gc.bf16_dev(v),
+                                          None if s is None else gc.to_dev(s), None if sinv is None else gc.to_dev(sinv),
+                                          status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    qz = oracle.quantize_all(q, k, v, s, sinv)
+    res = gc.oracle_from_gpu_layout_check(w, qq, kq, vq, qz)
+    assert all(res.values()), res
+
+
 def test_quantisers_bit_exact_full_qwen():
     w = configs.get("qwen3-8b-4k")
     q, k, v = gen.inputs(w)
