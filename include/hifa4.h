@@ -30,6 +30,8 @@
  *   - Shapes: d in {64, 128, 256}; Hq % Hkv == 0 (query head h uses kv head
  *     h / (Hq/Hkv)); N % 128 == 0; N <= 63488 (the FP16 normaliser stays finite); causal
  *     attention uses equal query and key lengths with key k visible to query i iff k <= i.
+ *     The FP16 running max holds RN(rowmax(S) * log2(e)/sqrt(d)); rows where that exceeds
+ *     the FP16 range (|.| > 65504) are outside the supported input range.
  *   - Requires an sm_100 device (B200); anything else returns
  *     HIFA4_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
  */

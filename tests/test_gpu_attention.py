@@ -32,11 +32,73 @@ def test_parity_reduced_all_rows(name, kw):
     gc.assert_parity(gc.run_parity(w))
 
 
-@pytest.mark.parametrize("name", ["tiny", "qwen3-8b-4k", "gemma2-9b-8k"])
+@pytest.mark.parametrize("name", configs.ORDER)
 def test_parity_full_size_sampled_rows(name):
+    # every workload at its full size; rows: the first and last 128-row query tile and 4
+    # seeded random rows of every (batch, head)
     w = configs.get(name)
     rows = gen.sample_rows(w, per_head=4) if w.N > 256 else None
     gc.assert_parity(gc.run_parity(w, rows, check_quant=False))
+
+
+EDGE = [
+    ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=128, bc=128)),                 # one query tile, one kv tile
+    ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=128, bc=128, causal=False)),
+    ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=256)),                         # 256-key tile, q-tile 0 half masked
+    ("qwen3-8b-4k", dict(Hq=4, Hkv=4, N=512)),                         # no GQA
+    ("llama3.1-8b-b4-16k", dict(B=3, Hq=2, Hkv=2, N=512, causal=False)),
+    ("gemma2-9b-8k", dict(B=2, Hq=2, Hkv=1, N=128)),                   # d = 256, two 64-key tiles
+]
+
+
+@pytest.mark.parametrize("name,kw", EDGE)
+def test_parity_edge_shapes(name, kw):
+    w = configs.scaled(configs.get(name), **kw)
+    gc.assert_parity(gc.run_parity(w))
+
+
+def _parity_custom(w, q, k, v, s=None, sinv=None, v_dev=None):
+    import oracle
+    qq, kq, vq, vt = gc.gpu_quantize(w, q, k, v, s, sinv)
+    qz = oracle.quantize_all(q, k, v, s, sinv)
+    res = gc.oracle_from_gpu_layout_check(w, qq, kq, vq, qz)
+    assert all(res.values()), res
+    o, m, l, code = gc.gpu_attention(w, qq, kq, vt if v_dev is None else v_dev)
+    assert code == hifa4.OK, hifa4.status_string(code)
+    rows = np.arange(w.B * w.Hq * w.N, dtype=np.int64)
+    ref = oracle.attn_fwd(qz, w.causal, w.bc, rows)
+    return gc.compare_outputs(w, rows, o, m, l, ref), o
+
+
+def test_zero_values_give_zero_output():
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=512)
+    q, k, v = gen.inputs(w)
+    stats, o = _parity_custom(w, q, k, np.zeros_like(v))
+    gc.assert_parity(stats)
+    assert float(o.float().abs().max()) == 0.0
+
+
+def test_large_and_widely_spread_scores():
+    # Q scaled by 8 and one K channel by 30: scores reach a few thousand (scaled max ~500,
+    # inside the FP16 range of m) and span far more than 127 in log2 units, so the exponent
+    # argument saturates and many blocks get the zero scale.
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=512)
+    q, k, v = gen.inputs(w)
+    qf = gen.bf16_bits_to_f32(q) * 8.0
+    kf = gen.bf16_bits_to_f32(k)
+    kf[..., 3] *= 30.0
+    stats, _ = _parity_custom(w, gen.f32_to_bf16_bits(qf), gen.f32_to_bf16_bits(kf), v)
+    gc.assert_parity(stats)
+
+
+def test_strided_value_input():
+    # V as a permuted view of a [B, N, H, d] buffer goes straight into hifa4_attn_fwd
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=4, Hkv=2, N=512)
+    q, k, v = gen.inputs(w)
+    v_view = gc.bf16_dev(np.ascontiguousarray(v.transpose(0, 2, 1, 3))).permute(0, 2, 1, 3)
+    assert not v_view.is_contiguous()
+    stats, _ = _parity_custom(w, q, k, v, v_dev=v_view)
+    gc.assert_parity(stats)
 
 
 def test_timeout_is_reported_and_context_survives():
