@@ -6,14 +6,16 @@
 // tensor core: an extra MMA of P_hat against a block of ones (N = 16) runs next to the
 // PV MMA, so no row sum of P is computed on the ALUs.
 //
-// One CTA works on one (batch, query head, 128-row query tile); kv tiles of BC keys are
+// Persistent kernel: one CTA per SM walks a list of work units (batch, query head, 128-row
+// query tile), longest first, in a snake order over the CTAs; kv tiles of BC keys are
 // visited in ascending order.  Warp roles:
-//   warp 0      TMA producer: Q tile once, then K and V^T tiles (+ their scale atoms)
-//               into KS / VS-deep shared-memory rings.
+//   warp 0      TMA producer: per unit the Q tile (double-buffered, so the next unit's Q
+//               arrives early), then K and V^T tiles (+ their scale atoms) into KS / VS-deep
+//               shared-memory rings.
 //   warp 1      allocates TMEM; lane 0 issues tcgen05.cp (scales -> TMEM) and MMAs:
-//               S_j = Q K_j^T into a double-buffered S, then O += P_hat_j V_j and
-//               R = P_hat_j * ones.
-//   warps 2..5  softmax: thread = one query row (TMEM lane).  Per tile: load S row, mask,
+//               S_j = Q K_j^T into the S buffers, then O += P_hat_j V_j and
+//               R = P_hat_j * ones.  The next unit's first QK^T overlaps the epilogue.
+//   warps 2..   softmax: thread = one query row (TMEM lane).  Per tile: load S row, mask,
 //               m_new = max(m, fp16(rowmax(S) * c)), P = E(fma(S, c, -m_new)) quantised to
 //               P_hat (codes -> shared memory in the MMA's swizzled layout, scales -> a
 //               scale atom), then after PV_{j-1} completed: l = fp16(fma(alpha_{j-1}, l,
@@ -45,21 +47,21 @@ struct AttnCfg {
   static constexpr uint32_t SZ_ONES = 16 * PROW;
   static constexpr uint32_t SZ_QSF = KQ * 512, SZ_KSF = NAK * KQ * 512, SZ_VSF = KP * NAV * 512, SZ_PSF = KP * 512;
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + align_up(SZ_Q, 1024);
+  static constexpr uint32_t OFF_K = OFF_Q + 2 * align_up(SZ_Q, 1024);
   static constexpr uint32_t OFF_V = OFF_K + KS * align_up(SZ_K, 1024);
   static constexpr uint32_t OFF_P = OFF_V + VS * align_up(SZ_V, 1024);
   static constexpr uint32_t OFF_ONES = OFF_P + 2 * align_up(SZ_P, 1024);
   static constexpr uint32_t OFF_QSF = OFF_ONES + align_up(SZ_ONES, 1024);
-  static constexpr uint32_t OFF_KSF = OFF_QSF + SZ_QSF;
+  static constexpr uint32_t OFF_KSF = OFF_QSF + 2 * SZ_QSF;
   static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
   static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
   static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 128 x fp32 table of L(sigma)
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
   static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 128 * 4;
-  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2],
-  // s_empty[2], p_full[2], o_bar, drain
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 6 + 2;
+  // barriers: q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
+  // s_full[2], s_empty[2], p_full[2], o_bar, o_free, drain
+  static constexpr int NBAR = 4 + 2 * KS + 2 * VS + 6 + 3;
   static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-B alignment
   // TMEM columns.  S is double-buffered when it fits; a single buffer is enough for
@@ -130,6 +132,22 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Work unit u (0 <= u < B*Hq*(N/128)) -> (batch*head, query tile); causal units are
+// ordered longest first (the last query tiles need the most kv tiles).
+__device__ __forceinline__ void unit_coords(int u, const AttnParams& p, int& bh, int& qtile) {
+  const int BH = p.B * p.Hq, nqt = p.N / 128;
+  qtile = p.causal ? nqt - 1 - u / BH : u / BH;
+  bh = u % BH;
+}
+
+template <int BC>
+__device__ __forceinline__ int unit_tiles(int qtile, const AttnParams& p) {
+  return p.causal ? ((qtile + 1) * 128 + BC - 1) / BC : p.N / BC;
+}
+
+// Persistent kernel: each CTA walks its share of the units (see unit_of).  Ring-buffer
+// phases run on a tile counter g that continues across units; the Q tile is
+// double-buffered so the next unit's Q arrives while the current one is processed.
 template <int D, int BC>
 __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -137,13 +155,12 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   using C = AttnCfg<D, BC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sOnes = smem + C::OFF_ONES;
-  uint8_t* sQsf = smem + C::OFF_QSF;
   uint8_t* s1sf = smem + C::OFF_1SF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* k_full = q_empty + 2;
   uint64_t* k_empty = k_full + C::KS;
   uint64_t* v_full = k_empty + C::KS;
   uint64_t* v_empty = v_full + C::VS;
@@ -151,9 +168,12 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* o_bar = p_full + 2;
-  uint64_t* drain_bar = o_bar + 1;
+  uint64_t* o_free = o_bar + 1;
+  uint64_t* drain_bar = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  auto sQ = [&](int s) { return smem + C::OFF_Q + s * align_up(C::SZ_Q, 1024); };
+  auto sQsf = [&](int s) { return smem + C::OFF_QSF + s * C::SZ_QSF; };
   auto sK = [&](int s) { return smem + C::OFF_K + s * align_up(C::SZ_K, 1024); };
   auto sV = [&](int s) { return smem + C::OFF_V + s * align_up(C::SZ_V, 1024); };
   auto sP = [&](int s) { return smem + C::OFF_P + s * align_up(C::SZ_P, 1024); };
@@ -162,19 +182,19 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   auto sPsf = [&](int s) { return smem + C::OFF_PSF + s * C::SZ_PSF; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.B * p.Hq;
   const int nqt = p.N / 128;
-  const int qtile = p.causal ? nqt - 1 - (int)(blockIdx.x / BH) : (int)(blockIdx.x / BH);
-  const int bh = blockIdx.x % BH;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
-  const int nt = p.causal ? ((qtile + 1) * 128 + BC - 1) / BC : p.N / BC;
+  const int units = p.B * p.Hq * nqt;
+  // the CTA's i-th unit: rows of gridDim.x units, every other row reversed (snake order),
+  // which evens out the per-CTA work of the longest-first causal list
+  auto unit_of = [&](int i) {
+    return i * (int)gridDim.x + ((i & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
       const bool per_warp = (&bars[i] == &s_empty[0] || &bars[i] == &s_empty[1] || &bars[i] == &p_full[0] ||
-                             &bars[i] == &p_full[1]);
-      mbar_init(&bars[i], per_warp ? 4 * C::NSW : 1);   // s_empty / p_full: one arrival per softmax warp
+                             &bars[i] == &p_full[1] || &bars[i] == o_free);
+      mbar_init(&bars[i], per_warp ? 4 * C::NSW : 1);   // one arrival per softmax warp
     }
     *abort = 0;
     fence_mbar_init();
@@ -204,57 +224,73 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(q_full, C::SZ_Q + C::SZ_QSF);
-      tma_load_2d(sQ, &tmQ, 0, bh * p.N + qtile * 128, q_full);
-      bulk_load(sQsf, p.qsf + ((long long)bh * nqt + qtile) * C::SZ_QSF, C::SZ_QSF, q_full);
-      int issued = 0;
-      for (int j = 0; j < nt; ++j) {
-        if (p.inject == 1 && j == 1) break;
-        const int ks = j % C::KS, vs = j % C::VS;
-        if (j >= C::KS && !mbar_wait(&k_empty[ks], ((j / C::KS) - 1) & 1, abort, p.status, p.wait_ns)) break;
-        mbar_arrive_expect_tx(&k_full[ks], C::SZ_K + C::SZ_KSF);
-        tma_load_2d(sK(ks), &tmK, 0, kvh * p.N + j * BC, &k_full[ks]);
-        const int katom = (j * BC) / 128;
-        // the tile's NAK consecutive 128-row atoms (KQ x 512 bytes each) are contiguous
-        bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * (C::KQ * 512), C::SZ_KSF, &k_full[ks]);
-        if (j >= C::VS && !mbar_wait(&v_empty[vs], ((j / C::VS) - 1) & 1, abort, p.status, p.wait_ns)) {
-          issued = 2 * j + 1;
-          break;
+      int nq = 0, nk = 0, nv = 0;   // loads issued (Q per unit, K and V per tile)
+      bool ok = true;
+      for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
+        int bh, qtile;
+        unit_coords(u, p, bh, qtile);
+        const int kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
+        const int nt = unit_tiles<BC>(qtile, p);
+        const int qb = i & 1;
+        if (i >= 2 && !mbar_wait(&q_empty[qb], ((i >> 1) - 1) & 1, abort, p.status, p.wait_ns)) break;
+        mbar_arrive_expect_tx(&q_full[qb], C::SZ_Q + C::SZ_QSF);
+        tma_load_2d(sQ(qb), &tmQ, 0, bh * p.N + qtile * 128, &q_full[qb]);
+        bulk_load(sQsf(qb), p.qsf + ((long long)bh * nqt + qtile) * C::SZ_QSF, C::SZ_QSF, &q_full[qb]);
+        ++nq;
+        for (int j = 0; j < nt; ++j) {
+          if (p.inject == 1 && i == 0 && j == 1) { ok = false; break; }
+          const int g = nk, ks = g % C::KS, vs = g % C::VS;
+          if (g >= C::KS && !mbar_wait(&k_empty[ks], ((g / C::KS) - 1) & 1, abort, p.status, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[ks], C::SZ_K + C::SZ_KSF);
+          tma_load_2d(sK(ks), &tmK, 0, kvh * p.N + j * BC, &k_full[ks]);
+          // the tile's NAK consecutive 128-row atoms (KQ x 512 bytes each) are contiguous
+          const int katom = (j * BC) / 128;
+          bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * (C::KQ * 512), C::SZ_KSF, &k_full[ks]);
+          ++nk;
+          if (g >= C::VS && !mbar_wait(&v_empty[vs], ((g / C::VS) - 1) & 1, abort, p.status, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[vs], C::SZ_V + C::SZ_VSF);
+          tma_load_2d(sV(vs), &tmV, j * C::PROW, kvh * D, &v_full[vs]);
+          bulk_load(sVsf(vs), p.vsf + ((long long)kvh * (p.N / 64) + j * C::KP) * (C::NAV * 512), C::SZ_VSF,
+                    &v_full[vs]);
+          ++nv;
         }
-        mbar_arrive_expect_tx(&v_full[vs], C::SZ_V + C::SZ_VSF);
-        tma_load_2d(sV(vs), &tmV, j * C::PROW, kvh * D, &v_full[vs]);
-        bulk_load(sVsf(vs), p.vsf + ((long long)kvh * (p.N / 64) + j * C::KP) * (C::NAV * 512), C::SZ_VSF,
-                  &v_full[vs]);
-        issued = 2 * j + 2;
       }
       // drain: every load this warp issued must have landed before the CTA exits
-      drain_wait(q_full, 0, p.status, p.wait_ns);
-      const int nk = (issued + 1) / 2, nv = issued / 2;
-      for (int s = 0; s < C::KS && s < nk; ++s) {
-        const int last = s + ((nk - 1 - s) / C::KS) * C::KS;
-        drain_wait(&k_full[s], (last / C::KS) & 1, p.status, p.wait_ns);
-      }
-      for (int s = 0; s < C::VS && s < nv; ++s) {
-        const int last = s + ((nv - 1 - s) / C::VS) * C::VS;
-        drain_wait(&v_full[s], (last / C::VS) & 1, p.status, p.wait_ns);
-      }
+      auto drain_ring = [&](uint64_t* full, int n, int stages) {
+        for (int s = 0; s < stages && s < n; ++s) {
+          const int last = s + ((n - 1 - s) / stages) * stages;
+          drain_wait(&full[s], (last / stages) & 1, p.status, p.wait_ns);
+        }
+      };
+      drain_ring(q_full, nq, 2);
+      drain_ring(k_full, nk, C::KS);
+      drain_ring(v_full, nv, C::VS);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t ID_QK = idesc_nvf4(128, BC), ID_PV = idesc_nvf4(128, D), ID_R = idesc_nvf4(128, 16);
-    const uint32_t aQ = smem_u32(sQ), aOnes = smem_u32(sOnes);
-    auto issue_pv = [&](int t) -> bool {
-      const int vs = t % C::VS, pb = t & 1;
-      bool ok = wait_all(&v_full[vs], (t / C::VS) & 1, abort, p.status, p.wait_ns);
-      ok = ok && wait_all(&p_full[pb], (t >> 1) & 1, abort, p.status, p.wait_ns);
+    const uint32_t aOnes = smem_u32(sOnes);
+    // PV of global tile g (local tile t of a unit processed as the CTA's i-th unit)
+    auto issue_pv = [&](int g, int t, int i) -> bool {
+      const int vs = g % C::VS, pb = g & 1;
+      bool ok = wait_all(&v_full[vs], (g / C::VS) & 1, abort, p.status, p.wait_ns);
+      ok = ok && wait_all(&p_full[pb], (g >> 1) & 1, abort, p.status, p.wait_ns);
+      // the previous unit's epilogue must have read O and R before they are overwritten
+      if (ok && t == 0 && i >= 1) ok = wait_all(o_free, (i - 1) & 1, abort, p.status, p.wait_ns);
       if (!ok) return false;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t sfv = tbase + C::T_SFV + pb * 4 * C::KP * C::NAV;
         const uint32_t sfp = tbase + C::T_SFP + pb * 4 * C::KP;
 #pragma unroll
-        for (int i = 0; i < C::KP * C::NAV; ++i) tmem_cp_sf_atom(sfv + 4 * i, sVsf(vs) + 512 * i);
+        for (int q = 0; q < C::KP * C::NAV; ++q) tmem_cp_sf_atom(sfv + 4 * q, sVsf(vs) + 512 * q);
 #pragma unroll
         for (int kc = 0; kc < C::KP; ++kc) tmem_cp_sf_atom(sfp + 4 * kc, sPsf(pb) + 512 * kc);
         const uint32_t aP = smem_u32(sP(pb)), aV = smem_u32(sV(vs));
@@ -274,54 +310,65 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       __syncwarp();
       return true;
     };
-    bool ok = wait_all(q_full, 0, abort, p.status, p.wait_ns);
-    if (ok) {
+    bool ok = true;
+    int g = 0;   // global tile counter
+    for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
+      int bh, qtile;
+      unit_coords(u, p, bh, qtile);
+      const int nt = unit_tiles<BC>(qtile, p);
+      const int qb = i & 1;
+      ok = wait_all(&q_full[qb], (i >> 1) & 1, abort, p.status, p.wait_ns);
+      // the previous unit's QK MMAs (which read the Q scale columns) have completed
+      if (ok && i >= 1) ok = wait_all(&q_empty[qb ^ 1], ((i - 1) >> 1) & 1, abort, p.status, p.wait_ns);
+      if (!ok) break;
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
-        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(tbase + C::T_SFQ + 4 * kc, sQsf + 512 * kc);
-        tmem_cp_sf_atom(tbase + C::T_SF1, s1sf);
+        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(tbase + C::T_SFQ + 4 * kc, sQsf(qb) + 512 * kc);
+        if (i == 0) tmem_cp_sf_atom(tbase + C::T_SF1, s1sf);
       }
       __syncwarp();
-    }
-    for (int j = 0; ok && j < nt; ++j) {
-      const int ks = j % C::KS, sb = j % C::SB;
-      ok = wait_all(&k_full[ks], (j / C::KS) & 1, abort, p.status, p.wait_ns);
-      if (ok && j >= C::SB) ok = wait_all(&s_empty[sb], ((j / C::SB) - 1) & 1, abort, p.status, p.wait_ns);
-      if (!ok) break;
-      if (BC == 64 && (j & 1)) {
-        // keys 64..127 of the 128-row scale atom: move record words 2,3 into words 0,1
+      const uint32_t aQ = smem_u32(sQ(qb));
+      for (int j = 0; ok && j < nt; ++j, ++g) {
+        const int ks = g % C::KS, sb = g % C::SB;
+        ok = wait_all(&k_full[ks], (g / C::KS) & 1, abort, p.status, p.wait_ns);
+        if (ok && g >= C::SB) ok = wait_all(&s_empty[sb], ((g / C::SB) - 1) & 1, abort, p.status, p.wait_ns);
+        if (!ok) break;
+        if (BC == 64 && (j & 1)) {
+          // keys 64..127 of the 128-row scale atom: move record words 2,3 into words 0,1
 #pragma unroll
-        for (int kc = 0; kc < C::KQ; ++kc) {
-          uint4* rec = reinterpret_cast<uint4*>(sKsf(ks) + 512 * kc) + lane;
-          uint4 w = *rec;
-          *rec = make_uint4(w.z, w.w, w.z, w.w);
+          for (int kc = 0; kc < C::KQ; ++kc) {
+            uint4* rec = reinterpret_cast<uint4*>(sKsf(ks) + 512 * kc) + lane;
+            uint4 w = *rec;
+            *rec = make_uint4(w.z, w.w, w.z, w.w);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      tc_fence_after();
-      if (lane == 0) {
-        // K scale atoms (row atom rt, chunk kc) -> 4 columns at chunk kc's 4*NAK columns + 4 rt
-        const uint32_t sfk = tbase + C::T_SFK + (j & 1) * 4 * C::KQ * C::NAK;
+        tc_fence_after();
+        if (lane == 0) {
+          // K scale atoms (row atom rt, chunk kc) -> 4 columns at chunk kc's 4*NAK columns + 4 rt
+          const uint32_t sfk = tbase + C::T_SFK + (g & 1) * 4 * C::KQ * C::NAK;
 #pragma unroll
-        for (int rt = 0; rt < C::NAK; ++rt)
+          for (int rt = 0; rt < C::NAK; ++rt)
+#pragma unroll
+            for (int kc = 0; kc < C::KQ; ++kc)
+              tmem_cp_sf_atom(sfk + 4 * (C::NAK * kc + rt), sKsf(ks) + 512 * (rt * C::KQ + kc));
+          const uint32_t aK = smem_u32(sK(ks));
 #pragma unroll
           for (int kc = 0; kc < C::KQ; ++kc)
-            tmem_cp_sf_atom(sfk + 4 * (C::NAK * kc + rt), sKsf(ks) + 512 * (rt * C::KQ + kc));
-        const uint32_t aK = smem_u32(sK(ks));
-#pragma unroll
-        for (int kc = 0; kc < C::KQ; ++kc)
-          mma_nvf4(tbase + C::T_S + sb * BC, smem_desc(aQ + 32 * kc, 0, 8 * C::QROW, C::LQ),
-                   smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc,
-                   sfk + 4 * C::NAK * kc, kc > 0 ? 1u : 0u);
-        tc_commit(&s_full[sb]);
-        tc_commit(&k_empty[ks]);
+            mma_nvf4(tbase + C::T_S + sb * BC, smem_desc(aQ + 32 * kc, 0, 8 * C::QROW, C::LQ),
+                     smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc,
+                     sfk + 4 * C::NAK * kc, kc > 0 ? 1u : 0u);
+          tc_commit(&s_full[sb]);
+          tc_commit(&k_empty[ks]);
+          if (j == nt - 1) tc_commit(&q_empty[qb]);   // the unit's Q tile and Q scales are free
+        }
+        __syncwarp();
+        if (j >= 1) ok = issue_pv(g - 1, j - 1, i);
       }
-      __syncwarp();
-      if (j >= 1) ok = issue_pv(j - 1);
+      if (ok) ok = issue_pv(g - 1, nt - 1, i);
     }
-    if (ok) ok = issue_pv(nt - 1);
     // drain: every MMA / copy this warp issued has completed before TMEM is freed
     if (lane == 0) {
       tc_commit(drain_bar);
@@ -330,140 +377,148 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps
-    // warp pairs (w, w+4) share TMEM lane quarter q4 (the same 32 query rows); warpgroup
+    // warps w, w+4, ... share TMEM lane quarter q4 (the same 32 query rows); warpgroup
     // wg takes score columns [wg*CW, wg*CW + CW) and O columns [wg*D/NSW, ...).
     constexpr int CW = C::CW, NB = CW / 16, OW = D / C::NSW;
     const int sw = warp - 2, wg = sw >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
-    const int qrow = qtile * 128 + row;
     const int col0 = wg * CW;
     const float c = p.c;
-    float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+    const float c7 = c * 0.0078125f;
     bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int sb = j % C::SB, pb = j & 1;
-      ok = wait_all(&s_full[sb], (j / C::SB) & 1, abort, p.status, p.wait_ns);
-      if (!ok) break;
-      tc_fence_after();
-      float s[CW];
-      {
-        uint32_t r[CW];
-#pragma unroll
-        for (int c0 = 0; c0 < CW; c0 += 32)
-          tmem_ld32(tbase + lrow + C::T_S + sb * BC + col0 + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
-        tmem_wait_ld();
-        reg_fence(r);
-#pragma unroll
-        for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(r[i]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[sb]);
-      if (p.causal && (j + 1) * BC - 1 > qtile * 128) {
-#pragma unroll
-        for (int i = 0; i < CW; ++i)
-          if (j * BC + col0 + i > qrow) s[i] = -INFINITY;
-      }
-      float bmax[NB];
-#pragma unroll
-      for (int bl = 0; bl < NB; ++bl) {
-        float m = s[bl * 16];
-#pragma unroll
-        for (int e = 1; e < 15; e += 2) m = fmax3(m, s[bl * 16 + e], s[bl * 16 + e + 1]);
-        bmax[bl] = fmaxf(m, s[bl * 16 + 15]);
-      }
-      float lmax = bmax[0];
-#pragma unroll
-      for (int bl = 1; bl < NB; ++bl) lmax = fmaxf(lmax, bmax[bl]);
-      // combine the partial row maxima of the NSW warpgroups (double-buffered by tile parity)
-      float* xm = xmax + (j & 1) * (C::NSW * 128);
-      xm[wg * 128 + row] = lmax;
-      named_bar(1 + q4, 32 * C::NSW);
-      float rmax = xm[row];
-#pragma unroll
-      for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
-      float mnew = m_run;
-      if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
-      // alpha = E(m - m_new): 0 on the first tile, exactly E(0) = 1 when the max is unchanged
-      const float alpha = (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
-      const float negm = -mnew;
-      const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
-      // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call
-      float pmax[NB];
-#pragma unroll
-      for (int bl = 0; bl < NB; bl += 2) {
-        const float2 e2 = exp2_own2(__ffma2_rn(make_float2(bmax[bl], bmax[bl + 1]), c2, negm2));
-        pmax[bl] = e2.x;
-        pmax[bl + 1] = e2.y;
-      }
-      const float c7 = c * 0.0078125f;
-      uint32_t words[CW / 8];
-      uint32_t sfw = 0;
-#pragma unroll
-      for (int bl = 0; bl < NB; ++bl) {
-        const uint32_t sc = cvt_e4m3(__fmul_rn(pmax[bl], kSixth));
-        sfw |= sc << (8 * bl);
-        // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-        const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
-#pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          float2 y[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = bl * 16 + h8 * 8 + 2 * k;
-            y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
-          }
-          words[2 * bl + h8] = encode8_pairs(y);
-        }
-      }
-      uint8_t* pbuf = sP(pb);
-#pragma unroll
-      for (int q = 0; q < CW / 32; ++q)
-        *reinterpret_cast<uint4*>(pbuf + swz_offset(row, col0 / 32 + q, C::PROW)) =
-            make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-      {
-        uint8_t* atom = sPsf(pb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
-        if (NB == 4) *reinterpret_cast<uint32_t*>(atom) = sfw;
-        else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
-      }
-      fence_proxy_async_smem();
-      if (j > 0) {
-        ok = wait_all(o_bar, (j - 1) & 1, abort, p.status, p.wait_ns);
+    int g = 0;   // global tile counter
+    for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
+      int bh, qtile;
+      unit_coords(u, p, bh, qtile);
+      const int nt = unit_tiles<BC>(qtile, p);
+      const int qrow = qtile * 128 + row;
+      float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+      for (int j = 0; j < nt; ++j, ++g) {
+        const int sb = g % C::SB, pb = g & 1;
+        ok = wait_all(&s_full[sb], (g / C::SB) & 1, abort, p.status, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
-        uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
-        tmem_wait_ld();
-        reg_fence(rr);
-        l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll 1
-          for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tbase + lrow + C::T_O + c0, o);
-            tmem_wait_ld();
-            reg_fence(o);
-            const float2 a2 = make_float2(alpha, alpha);
+        float s[CW];
+        {
+          uint32_t r[CW];
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2);
-              o[i] = __float_as_uint(v.x);
-              o[i + 1] = __float_as_uint(v.y);
-            }
-            tmem_st32(tbase + lrow + C::T_O + c0, o);
-          }
-          tmem_wait_st();
+          for (int c0 = 0; c0 < CW; c0 += 32)
+            tmem_ld32(tbase + lrow + C::T_S + sb * BC + col0 + c0, *reinterpret_cast<uint32_t(*)[32]>(&r[c0]));
+          tmem_wait_ld();
+          reg_fence(r);
+#pragma unroll
+          for (int q = 0; q < CW; ++q) s[q] = __uint_as_float(r[q]);
         }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[sb]);
+        if (p.causal && (j + 1) * BC - 1 > qtile * 128) {
+#pragma unroll
+          for (int q = 0; q < CW; ++q)
+            if (j * BC + col0 + q > qrow) s[q] = -INFINITY;
+        }
+        float bmax[NB];
+#pragma unroll
+        for (int bl = 0; bl < NB; ++bl) {
+          float m = s[bl * 16];
+#pragma unroll
+          for (int e = 1; e < 15; e += 2) m = fmax3(m, s[bl * 16 + e], s[bl * 16 + e + 1]);
+          bmax[bl] = fmaxf(m, s[bl * 16 + 15]);
+        }
+        float lmax = bmax[0];
+#pragma unroll
+        for (int bl = 1; bl < NB; ++bl) lmax = fmaxf(lmax, bmax[bl]);
+        // combine the partial row maxima of the NSW warpgroups (double-buffered by parity)
+        float* xm = xmax + (g & 1) * (C::NSW * 128);
+        xm[wg * 128 + row] = lmax;
+        named_bar(1 + q4, 32 * C::NSW);
+        float rmax = xm[row];
+#pragma unroll
+        for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
+        float mnew = m_run;
+        if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
+        // alpha = E(m - m_new): 0 on the first tile, exactly E(0) = 1 when the max is unchanged
+        const float alpha =
+            (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
+        const float negm = -mnew;
+        const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
+        // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call
+        float pmax[NB];
+#pragma unroll
+        for (int bl = 0; bl < NB; bl += 2) {
+          const float2 e2 = exp2_own2(__ffma2_rn(make_float2(bmax[bl], bmax[bl + 1]), c2, negm2));
+          pmax[bl] = e2.x;
+          pmax[bl + 1] = e2.y;
+        }
+        uint32_t words[CW / 8];
+        uint32_t sfw = 0;
+#pragma unroll
+        for (int bl = 0; bl < NB; ++bl) {
+          const uint32_t sc = cvt_e4m3(__fmul_rn(pmax[bl], kSixth));
+          sfw |= sc << (8 * bl);
+          // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
+          const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
+#pragma unroll
+          for (int h8 = 0; h8 < 2; ++h8) {
+            float2 y[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = bl * 16 + h8 * 8 + 2 * k;
+              y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
+            }
+            words[2 * bl + h8] = encode8_pairs(y);
+          }
+        }
+        uint8_t* pbuf = sP(pb);
+#pragma unroll
+        for (int q = 0; q < CW / 32; ++q)
+          *reinterpret_cast<uint4*>(pbuf + swz_offset(row, col0 / 32 + q, C::PROW)) =
+              make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
+        {
+          uint8_t* atom = sPsf(pb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
+          if (NB == 4) *reinterpret_cast<uint32_t*>(atom) = sfw;
+          else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
+        }
+        fence_proxy_async_smem();
+        if (j > 0) {
+          ok = wait_all(o_bar, (g - 1) & 1, abort, p.status, p.wait_ns);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
+          tmem_wait_ld();
+          reg_fence(rr);
+          l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+            for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tbase + lrow + C::T_O + c0, o);
+              tmem_wait_ld();
+              reg_fence(o);
+              const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+              for (int q = 0; q < 32; q += 2) {
+                const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[q]), __uint_as_float(o[q + 1])), a2);
+                o[q] = __float_as_uint(v.x);
+                o[q + 1] = __float_as_uint(v.y);
+              }
+              tmem_st32(tbase + lrow + C::T_O + c0, o);
+            }
+            tmem_wait_st();
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[pb]);
+        alpha_prev = alpha;
+        m_run = mnew;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[pb]);
-      alpha_prev = alpha;
-      m_run = mnew;
-    }
-    if (ok) ok = wait_all(o_bar, (nt - 1) & 1, abort, p.status, p.wait_ns);
-    if (ok) {
+      if (!ok) break;
+      // epilogue: read R and O of the unit's last PV, release them, then O / l -> bf16
+      ok = wait_all(o_bar, (g - 1) & 1, abort, p.status, p.wait_ns);
+      if (!ok) break;
       tc_fence_after();
       uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
       tmem_wait_ld();
@@ -478,12 +533,18 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         tmem_ld32(tbase + lrow + C::T_O + c0, o);
         tmem_wait_ld();
         reg_fence(o);
+        if (c0 + 32 == wg * OW + OW) {
+          // every TMEM read of this unit is done: the next unit's first PV may overwrite O, R
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * i]), inv),
-                                                    __fmul_rn(__uint_as_float(o[2 * i + 1]), inv));
-          pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+        for (int q = 0; q < 16; ++q) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * q]), inv),
+                                                    __fmul_rn(__uint_as_float(o[2 * q + 1]), inv));
+          pk[q] = *reinterpret_cast<uint32_t*>(&v2);
         }
 #pragma unroll
         for (int q = 0; q < 4; ++q) dst[c0 / 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);

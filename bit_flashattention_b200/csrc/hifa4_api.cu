@@ -166,7 +166,17 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   p.wait_ns = g_wait_ns;
   p.inject = g_inject;
   fill_neg_log2_scales(p.lneg);
-  const unsigned grid = (unsigned)(B * Hq * (N / 128));
+  // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM)
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC>, C::NTHREADS, smem) != cudaSuccess ||
+        n <= 0)
+      n = 1;
+    per_sm = n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
+  }
+  const long long units = (long long)B * Hq * (N / 128), cap = (long long)per_sm * num_sms();
+  const unsigned grid = (unsigned)(units < cap ? units : cap);
   k_attn_fwd<D, BC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
