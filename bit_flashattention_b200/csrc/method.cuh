@@ -52,17 +52,16 @@ __device__ __forceinline__ float2 exp2_own2(float2 x) {
   return make_float2(insert_exponent(p.x, v.x), insert_exponent(p.y, v.y));
 }
 
-// P_hat evaluation in the log domain.  With the per-block bias B = (L(sigma) - m + 125)/128,
-// L(sigma) = RN(-log2 sigma), a score's u = sat(S * c/128 + B) and
-//   y = p(frac(128 u)) * 2^(floor(128 u) - 125)  ~  2^(S c - m) / sigma,
-// the value whose E2M1 rounding is the score's P_hat code.  The floor comes from a
-// round-down add of kPhatMagic (1.5 * 2^16 plus 387 ulps of 2^-7): its low mantissa bits
-// then hold floor(128 u) + 387, and 387 = -125 mod 512, so bits(v) << 23 is already the
-// exponent offset floor(128 u) - 125.  The polynomial runs on d = u - floor(128 u)/128
-// with coefficients scaled by 128 and 128^2, which rounds exactly as p on f = 128 d.
-constexpr float kPhatMagic = 98307.0234375f;          // 0x47C00183
-constexpr float kPhatC1 = kExp2C1 * 128.0f;
-constexpr float kPhatC2 = kExp2C2 * 16384.0f;
+// P_hat code decision in the log domain.  With the per-block bias
+// B = (L(sigma) - m + 125)/128, L(sigma) = RN(-log2 sigma), a score's u = sat(S * c/128 + B)
+// holds log2(P / sigma) + 125 scaled into [0, 1].  The code is the E2M1 rounding of the
+// linear-mantissa exponential y = 2^floor(z) * (1 + frac z) of z = 128 u - 125 + delta on a
+// 2^-10 grid (delta = -73/1024 centres the E2M1 rounding boundaries on those of the exact
+// exponential).  One fma forms v = 128 u + kPhatM, kPhatM = 8194 + delta: v lies in
+// [2^13, 2^14), whose spacing is 2^-10, so v's mantissa field is (z + 127) * 2^10, and
+// shifting v's bits left by 13 leaves exactly the bits of y (exponent floor(z) + 127, top
+// ten mantissa bits frac z).
+constexpr float kPhatM = 8193.9287109375f;   // 8194 - 73/1024
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   float d;
@@ -71,13 +70,8 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
 }
 
 __device__ __forceinline__ float2 phat_pair(float2 u) {
-  const float2 v = __fadd2_rd(u, make_float2(kPhatMagic, kPhatMagic));
-  const float2 w = __fadd2_rn(v, make_float2(-kPhatMagic, -kPhatMagic));
-  const float2 d = __ffma2_rn(w, make_float2(-1.0f, -1.0f), u);          // u - w, exact
-  float2 p = __ffma2_rn(make_float2(kPhatC2, kPhatC2), d, make_float2(kPhatC1, kPhatC1));
-  p = __ffma2_rn(p, d, make_float2(1.0f, 1.0f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(v.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(v.y) << 23)));
+  const float2 v = __ffma2_rn(u, make_float2(128.0f, 128.0f), make_float2(kPhatM, kPhatM));
+  return make_float2(__uint_as_float(__float_as_uint(v.x) << 13), __uint_as_float(__float_as_uint(v.y) << 13));
 }
 
 // Eight values held as four pairs (element 2k in .x) -> eight E2M1 codes, low nibble first.

@@ -24,7 +24,8 @@
  *     P = E(RN(fma(S, c, -m_new))), alpha = E(RN(m_old - m_new)),
  *     a block's scale sigma comes from E(fma(blockmax(S), c, -m_new)) (equal to the block
  *     amax of P because E is monotone -- pinned by a test), and a score's P_hat code is
- *     the E2M1 rounding of P/sigma evaluated in the log domain (phat_value()),
+ *     the E2M1 rounding of P/sigma evaluated in the log domain with a linear mantissa
+ *     (phat_value()),
  *     l = fp16_RN(fma(alpha, l, r)), r = exact sum of the tile's P_hat,
  *     O = alpha*O (fp32) + (exact tile P_hat V_hat rounded to fp32),
  *     out = bf16_RN(RN(O / l)).
@@ -153,19 +154,26 @@ static float neg_log2_scale(uint8_t code) {
 }
 
 /* The value whose E2M1 rounding is the P_hat code of a score: P / sigma evaluated in the
- * log domain.  Per block, B = RN(RN(L(sigma) - m) + 125) / 128; per score,
- * u = min(1, max(0, RN(S * (c/128) + B)))   (NaN -> 0), k = floor(128 u), f = 128 u - k,
- * y = p(f) * 2^(k - 125) with the exp2 polynomial p, i.e. y ~ 2^(S c - m) / sigma with the
- * exponent argument held in [-125, 3] (outside it every code is already 0 or saturated). */
+ * log domain with a linear mantissa.  Per block, B = RN(RN(L(sigma) - m) + 125) / 128;
+ * per score
+ *   u = min(1, max(0, RN(S * (c/128) + B)))          (NaN -> 0)
+ *   z = 128 u - 125 + DELTA, rounded to a multiple of 2^-10 (round to nearest even)
+ *   y = 2^floor(z) * (1 + z - floor(z)).
+ * 128 u - 125 is log2(P / sigma) = S c - m - log2(sigma) held in [-125, 3]; y is the
+ * piecewise-linear (linear-mantissa) exponential of z.  Only the E2M1 code of y is used,
+ * and that code changes where y crosses 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5: with
+ * DELTA = -73/1024 those crossings lie within 0.014 (log2 units) of the crossings of the
+ * exact 2^(S c - m) / sigma, except the crossing at 0.25 (codes 0 and 1), which lies 0.071
+ * above it.  Outside [-125, 3] every code is already 0 or saturated. */
+#define PHAT_DELTA (-73.0 / 1024.0)
 static float phat_value(float S, float c, float B) {
     float u = fmaf(S, c * 0.0078125f, B);
     if (!(u > 0.0f)) u = 0.0f;
     if (u > 1.0f) u = 1.0f;
-    float x = u * 128.0f;                 /* exact */
-    float k = floorf(x);
-    float f = x - k;                      /* exact */
-    float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);
-    return ldexpf(p, (int)k - 125);       /* exact: p in [1,2), result normal */
+    double t = (double)u * 128.0 - 125.0 + PHAT_DELTA;   /* exact: u has 24 bits */
+    double z = nearbyint(t * 1024.0) / 1024.0;           /* round half to even */
+    double k = floor(z);
+    return (float)ldexp(1.0 + (z - k), (int)k);          /* exact: 11 significant bits */
 }
 
 /* ------------------------------------------------------------------ block quantiser */
