@@ -12,10 +12,11 @@
 //   warp 0      TMA producer: per unit the Q tile (double-buffered, so the next unit's Q
 //               arrives early), then K and V^T tiles (+ their scale atoms) into KS / VS-deep
 //               shared-memory rings.
-//   warp 1      allocates TMEM; lane 0 issues tcgen05.cp (scales -> TMEM) and MMAs:
-//               S_j = Q K_j^T into the S buffers, then O += P_hat_j V_j and
-//               R = P_hat_j * ones.  The next unit's first QK^T overlaps the epilogue.
-//   warps 2..   softmax: thread = one query row (TMEM lane).  Per tile: load S row, mask,
+//   warp 1      allocates TMEM; issues tcgen05.cp (Q, K scales -> TMEM) and the QK^T MMAs
+//               S_j = Q K_j^T into the S buffers.  The next unit's first QK^T overlaps the
+//               epilogue.
+//   warp 2      issues the PV MMAs: O (+)= P_hat_j V_j and R = P_hat_j * ones.
+//   warps 3..   softmax: thread = one query row (TMEM lane).  Per tile: load S row, mask,
 //               m_new = max(m, fp16(rowmax(S) * c)), P = E(fma(S, c, -m_new)) quantised to
 //               P_hat (codes -> shared memory in the MMA's swizzled layout, scales -> a
 //               scale atom), then after PV_{j-1} completed: l = fp16(fma(alpha_{j-1}, l,
@@ -60,8 +61,8 @@ struct AttnCfg {
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
   static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 128 * 4;
   // barriers: q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
-  // s_full[2], s_empty[2], p_full[2], o_bar, o_free, drain
-  static constexpr int NBAR = 4 + 2 * KS + 2 * VS + 6 + 3;
+  // s_full[2], s_empty[2], p_full[2], o_bar, o_free, drain[2]
+  static constexpr int NBAR = 4 + 2 * KS + 2 * VS + 6 + 4;
   static constexpr uint32_t OFF_MISC = OFF_BAR + 8 * NBAR;
   static constexpr uint32_t SMEM = OFF_MISC + 16 + 1024;   // + slack for 1024-B alignment
   // TMEM columns.  S is double-buffered when it fits; a single buffer is enough for
@@ -84,7 +85,7 @@ struct AttnCfg {
   static constexpr int NSW = NSW0 < HIFA4_MAX_NSW ? NSW0 : HIFA4_MAX_NSW, CW = BC / NSW;
   static_assert(NSW == 2 || NSW == 4, "softmax warpgroups");
   static_assert(CW == 32 || CW == 64, "column split");
-  static constexpr int NTHREADS = 64 + 128 * NSW;
+  static constexpr int NTHREADS = 96 + 128 * NSW;   // producer, QK^T issuer, PV issuer, softmax
 };
 
 struct AttnParams {
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   uint64_t* p_full = s_empty + 2;
   uint64_t* o_bar = p_full + 2;
   uint64_t* o_free = o_bar + 1;
-  uint64_t* drain_bar = o_free + 1;
+  uint64_t* drain_bar = o_free + 1;   // [0] QK^T issuer, [1] PV issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   auto sQ = [&](int s) { return smem + C::OFF_Q + s * align_up(C::SZ_Q, 1024); };
@@ -201,9 +202,9 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   }
   float* rtab = reinterpret_cast<float*>(smem + C::OFF_RTAB);
   float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
-  if (warp >= 2) {
+  if (warp >= 3) {
     // the ones operand (E2M1 1.0 = 0b0010 in both nibbles) and its scales (UE4M3 1.0)
-    const int t = threadIdx.x - 64, nt2 = 128 * C::NSW;
+    const int t = threadIdx.x - 96, nt2 = 128 * C::NSW;
     for (int i = t; i < (int)C::SZ_ONES / 4; i += nt2) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
     for (int i = t; i < 128; i += nt2) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
     fence_proxy_async_smem();
@@ -274,42 +275,14 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t ID_QK = idesc_nvf4(128, BC), ID_PV = idesc_nvf4(128, D), ID_R = idesc_nvf4(128, 16);
-    const uint32_t aOnes = smem_u32(sOnes);
-    // PV of global tile g (local tile t of a unit processed as the CTA's i-th unit)
-    auto issue_pv = [&](int g, int t, int i) -> bool {
-      const int vs = g % C::VS, pb = g & 1;
-      bool ok = wait_all(&v_full[vs], (g / C::VS) & 1, abort, p.status, p.wait_ns);
-      ok = ok && wait_all(&p_full[pb], (g >> 1) & 1, abort, p.status, p.wait_ns);
-      // the previous unit's epilogue must have read O and R before they are overwritten
-      if (ok && t == 0 && i >= 1) ok = wait_all(o_free, (i - 1) & 1, abort, p.status, p.wait_ns);
-      if (!ok) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t sfv = tbase + C::T_SFV + pb * 4 * C::KP * C::NAV;
-        const uint32_t sfp = tbase + C::T_SFP + pb * 4 * C::KP;
-#pragma unroll
-        for (int q = 0; q < C::KP * C::NAV; ++q) tmem_cp_sf_atom(sfv + 4 * q, sVsf(vs) + 512 * q);
-#pragma unroll
-        for (int kc = 0; kc < C::KP; ++kc) tmem_cp_sf_atom(sfp + 4 * kc, sPsf(pb) + 512 * kc);
-        const uint32_t aP = smem_u32(sP(pb)), aV = smem_u32(sV(vs));
-#pragma unroll
-        for (int kc = 0; kc < C::KP; ++kc)
-          mma_nvf4(tbase + C::T_O, smem_desc(aP + 32 * kc, 0, 8 * C::PROW, C::LP),
-                   smem_desc(aV + 32 * kc, 0, 8 * C::PROW, C::LP), ID_PV, sfp + 4 * kc, sfv + 4 * C::NAV * kc,
-                   (t > 0 || kc > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kc = 0; kc < C::KP; ++kc)
-          mma_nvf4(tbase + C::T_R, smem_desc(aP + 32 * kc, 0, 8 * C::PROW, C::LP),
-                   smem_desc(aOnes + 32 * kc, 0, 8 * C::PROW, C::LP), ID_R, sfp + 4 * kc, tbase + C::T_SF1,
-                   kc > 0 ? 1u : 0u);
-        tc_commit(o_bar);
-        tc_commit(&v_empty[vs]);
-      }
-      __syncwarp();
-      return true;
-    };
+    // ------------------------------------------------------------ QK^T issuer
+    // S_g = Q K_g^T into S buffer g % SB.  Shared-memory descriptors are formed once; a
+    // byte offset inside the (256 KB) window adds offset >> 4 to the start-address field.
+    constexpr uint32_t ID_QK = idesc_nvf4(128, BC);
+    const uint64_t dQ = smem_desc(smem_u32(sQ(0)), 0, 8 * C::QROW, C::LQ);
+    const uint64_t dK = smem_desc(smem_u32(sK(0)), 0, 8 * C::QROW, C::LQ);
+    const uint64_t dQsf = smem_desc(smem_u32(sQsf(0)), 0, 128, 0);
+    const uint64_t dKsf = smem_desc(smem_u32(sKsf(0)), 0, 128, 0);
     bool ok = true;
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
@@ -324,11 +297,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       tc_fence_after();
       if (lane == 0) {
 #pragma unroll
-        for (int kc = 0; kc < C::KQ; ++kc) tmem_cp_sf_atom(tbase + C::T_SFQ + 4 * kc, sQsf(qb) + 512 * kc);
-        if (i == 0) tmem_cp_sf_atom(tbase + C::T_SF1, s1sf);
+        for (int kc = 0; kc < C::KQ; ++kc)
+          tmem_cp_sf(tbase + C::T_SFQ + 4 * kc, dQsf + ((qb * C::SZ_QSF + 512 * kc) >> 4));
       }
       __syncwarp();
-      const uint32_t aQ = smem_u32(sQ(qb));
+      const uint64_t dQi = dQ + ((qb * align_up(C::SZ_Q, 1024)) >> 4);
       for (int j = 0; ok && j < nt; ++j, ++g) {
         const int ks = g % C::KS, sb = g % C::SB;
         ok = wait_all(&k_full[ks], (g / C::KS) & 1, abort, p.status, p.wait_ns);
@@ -349,30 +322,84 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         if (lane == 0) {
           // K scale atoms (row atom rt, chunk kc) -> 4 columns at chunk kc's 4*NAK columns + 4 rt
           const uint32_t sfk = tbase + C::T_SFK + (g & 1) * 4 * C::KQ * C::NAK;
+          const uint64_t dKsfs = dKsf + ((ks * C::SZ_KSF) >> 4);
 #pragma unroll
           for (int rt = 0; rt < C::NAK; ++rt)
 #pragma unroll
             for (int kc = 0; kc < C::KQ; ++kc)
-              tmem_cp_sf_atom(sfk + 4 * (C::NAK * kc + rt), sKsf(ks) + 512 * (rt * C::KQ + kc));
-          const uint32_t aK = smem_u32(sK(ks));
+              tmem_cp_sf(sfk + 4 * (C::NAK * kc + rt), dKsfs + ((512 * (rt * C::KQ + kc)) >> 4));
+          const uint64_t dKs = dK + ((ks * align_up(C::SZ_K, 1024)) >> 4);
 #pragma unroll
           for (int kc = 0; kc < C::KQ; ++kc)
-            mma_nvf4(tbase + C::T_S + sb * BC, smem_desc(aQ + 32 * kc, 0, 8 * C::QROW, C::LQ),
-                     smem_desc(aK + 32 * kc, 0, 8 * C::QROW, C::LQ), ID_QK, tbase + C::T_SFQ + 4 * kc,
+            mma_nvf4(tbase + C::T_S + sb * BC, dQi + 2 * kc, dKs + 2 * kc, ID_QK, tbase + C::T_SFQ + 4 * kc,
                      sfk + 4 * C::NAK * kc, kc > 0 ? 1u : 0u);
           tc_commit(&s_full[sb]);
           tc_commit(&k_empty[ks]);
           if (j == nt - 1) tc_commit(&q_empty[qb]);   // the unit's Q tile and Q scales are free
         }
         __syncwarp();
-        if (j >= 1) ok = issue_pv(g - 1, j - 1, i);
       }
-      if (ok) ok = issue_pv(g - 1, nt - 1, i);
     }
     // drain: every MMA / copy this warp issued has completed before TMEM is freed
     if (lane == 0) {
-      tc_commit(drain_bar);
-      drain_wait(drain_bar, 0, p.status, p.wait_ns);
+      tc_commit(&drain_bar[0]);
+      drain_wait(&drain_bar[0], 0, p.status, p.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ PV issuer
+    // O (+)= P_hat_g V_g and R = P_hat_g * ones, once the softmax warps have written
+    // P_hat_g and applied alpha to O (p_full).
+    constexpr uint32_t ID_PV = idesc_nvf4(128, D), ID_R = idesc_nvf4(128, 16);
+    const uint64_t dP = smem_desc(smem_u32(sP(0)), 0, 8 * C::PROW, C::LP);
+    const uint64_t dV = smem_desc(smem_u32(sV(0)), 0, 8 * C::PROW, C::LP);
+    const uint64_t dOnes = smem_desc(smem_u32(sOnes), 0, 8 * C::PROW, C::LP);
+    const uint64_t dPsf = smem_desc(smem_u32(sPsf(0)), 0, 128, 0);
+    const uint64_t dVsf = smem_desc(smem_u32(sVsf(0)), 0, 128, 0);
+    tc_fence_after();
+    if (lane == 0) tmem_cp_sf(tbase + C::T_SF1, smem_desc(smem_u32(s1sf), 0, 128, 0));
+    __syncwarp();
+    bool ok = true;
+    int g = 0;   // global tile counter
+    for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
+      int bh, qtile;
+      unit_coords(u, p, bh, qtile);
+      const int nt = unit_tiles<BC>(qtile, p);
+      for (int j = 0; ok && j < nt; ++j, ++g) {
+        const int vs = g % C::VS, pb = g & 1;
+        ok = wait_all(&v_full[vs], (g / C::VS) & 1, abort, p.status, p.wait_ns);
+        ok = ok && wait_all(&p_full[pb], (g >> 1) & 1, abort, p.status, p.wait_ns);
+        // the previous unit's epilogue must have read O and R before they are overwritten
+        if (ok && j == 0 && i >= 1) ok = wait_all(o_free, (i - 1) & 1, abort, p.status, p.wait_ns);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t sfv = tbase + C::T_SFV + pb * 4 * C::KP * C::NAV;
+          const uint32_t sfp = tbase + C::T_SFP + pb * 4 * C::KP;
+          const uint64_t dVsfs = dVsf + ((vs * C::SZ_VSF) >> 4), dPsfs = dPsf + ((pb * C::SZ_PSF) >> 4);
+#pragma unroll
+          for (int q = 0; q < C::KP * C::NAV; ++q) tmem_cp_sf(sfv + 4 * q, dVsfs + 32 * q);
+#pragma unroll
+          for (int kc = 0; kc < C::KP; ++kc) tmem_cp_sf(sfp + 4 * kc, dPsfs + 32 * kc);
+          const uint64_t dPs = dP + ((pb * align_up(C::SZ_P, 1024)) >> 4);
+          const uint64_t dVs = dV + ((vs * align_up(C::SZ_V, 1024)) >> 4);
+#pragma unroll
+          for (int kc = 0; kc < C::KP; ++kc)
+            mma_nvf4(tbase + C::T_O, dPs + 2 * kc, dVs + 2 * kc, ID_PV, sfp + 4 * kc, sfv + 4 * C::NAV * kc,
+                     (j > 0 || kc > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kc = 0; kc < C::KP; ++kc)
+            mma_nvf4(tbase + C::T_R, dPs + 2 * kc, dOnes + 2 * kc, ID_R, sfp + 4 * kc, tbase + C::T_SF1,
+                     kc > 0 ? 1u : 0u);
+          tc_commit(o_bar);
+          tc_commit(&v_empty[vs]);
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) {
+      tc_commit(&drain_bar[1]);
+      drain_wait(&drain_bar[1], 0, p.status, p.wait_ns);
     }
     __syncwarp();
   } else {
@@ -380,7 +407,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     // warps w, w+4, ... share TMEM lane quarter q4 (the same 32 query rows); warpgroup
     // wg takes score columns [wg*CW, wg*CW + CW) and O columns [wg*D/NSW, ...).
     constexpr int CW = C::CW, NB = CW / 16, OW = D / C::NSW;
-    const int sw = warp - 2, wg = sw >> 2;
+    const int sw = warp - 3, wg = sw >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
