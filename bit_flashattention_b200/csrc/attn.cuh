@@ -414,7 +414,46 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     const int col0 = wg * CW;
     const float c = p.c;
     const float c7 = c * 0.0078125f;
+    // Epilogue of a unit whose last tile is gl: read R and O of that tile's PV, release
+    // them (o_free), then O / l -> bf16.  It runs after the next unit's first tile, which
+    // touches neither O nor R, so that tile's work overlaps the last PV.
+    auto epilogue = [&](int gl, long long orow, float l_e, float alpha_e) -> bool {
+      if (!wait_all(o_bar, gl & 1, abort, p.status, p.wait_ns)) return false;
+      tc_fence_after();
+      uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
+      tmem_wait_ld();
+      reg_fence(rr);
+      const float l_fin = f16_round(__fmaf_rn(alpha_e, l_e, __uint_as_float(rr[0])));
+      const float inv = (l_fin > 0.0f) ? __frcp_rn(l_fin) : 0.0f;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
+#pragma unroll 1
+      for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tbase + lrow + C::T_O + c0, o);
+        tmem_wait_ld();
+        reg_fence(o);
+        if (c0 + 32 == wg * OW + OW) {
+          // every TMEM read of this unit is done: the next unit's first PV may overwrite O, R
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(o_free);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * q]), inv),
+                                                    __fmul_rn(__uint_as_float(o[2 * q + 1]), inv));
+          pk[q] = *reinterpret_cast<uint32_t*>(&v2);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[c0 / 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      if (wg == 0 && p.l_out) p.l_out[orow] = __float2half_rn(l_fin);
+      return true;
+    };
     bool ok = true;
+    long long pend_row = 0;                  // the previous unit's output row, l and alpha
+    float pend_l = 0.0f, pend_alpha = 0.0f;
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
       int bh, qtile;
@@ -541,46 +580,18 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[pb]);
         alpha_prev = alpha;
         m_run = mnew;
+        if (j == 0 && i > 0) {
+          ok = epilogue(g - 1, pend_row, pend_l, pend_alpha);
+          if (!ok) break;
+        }
       }
       if (!ok) break;
-      // epilogue: read R and O of the unit's last PV, release them, then O / l -> bf16
-      ok = wait_all(o_bar, (g - 1) & 1, abort, p.status, p.wait_ns);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
-      tmem_wait_ld();
-      reg_fence(rr);
-      l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
-      const float inv = (l_run > 0.0f) ? __frcp_rn(l_run) : 0.0f;
-      const long long orow = (long long)bh * p.N + qrow;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
-#pragma unroll 1
-      for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tbase + lrow + C::T_O + c0, o);
-        tmem_wait_ld();
-        reg_fence(o);
-        if (c0 + 32 == wg * OW + OW) {
-          // every TMEM read of this unit is done: the next unit's first PV may overwrite O, R
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(o[2 * q]), inv),
-                                                    __fmul_rn(__uint_as_float(o[2 * q + 1]), inv));
-          pk[q] = *reinterpret_cast<uint32_t*>(&v2);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) dst[c0 / 8 + q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-      }
-      if (wg == 0) {
-        if (p.m_out) p.m_out[orow] = __float2half_rn(m_run);
-        if (p.l_out) p.l_out[orow] = __float2half_rn(l_run);
-      }
+      pend_row = (long long)bh * p.N + qrow;
+      pend_l = l_run;
+      pend_alpha = alpha_prev;
+      if (wg == 0 && p.m_out) p.m_out[pend_row] = __float2half_rn(m_run);
     }
+    if (ok && g > 0) ok = epilogue(g - 1, pend_row, pend_l, pend_alpha);
   }
   tc_fence_before();
   __syncthreads();
