@@ -27,6 +27,10 @@ if ROOT not in sys.path:
 WORKLOAD = "qwen3-8b-4k"
 N_SETS = 6                      # rotated input sets: 6 x ~50 MB of bf16 inputs > 126 MB L2
 FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
+# DRAM bytes (read + write) of one k_attn_fwd<128, 256> launch on qwen3-8b-4k, from an ncu
+# capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum; summary and
+# command in profiles/attn_fwd_qwen3-8b-4k.md).  Set to None when the kernel changes.
+ATTN_TRAFFIC_BYTES = 14.216e6 + 0.072e6
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 
@@ -237,6 +241,9 @@ def run_gpu(args):
     hbm, bf16, src = peaks()
     fp4_peak = bf16 * FP4_OVER_BF16
     achieved = flops / (k_attn * 1e-3) / 1e12
+    # algorithmic HBM bytes of one attention launch: 4-bit Q, K, V^T (codes + scales) read,
+    # bf16 O and fp16 m, l written
+    attn_bytes = B * (Hq + 2 * Hkv) * N * d * (0.5 + 1 / 16) + B * Hq * N * (2 * d + 4)
     quant_bytes = (B * (Hq + 2 * Hkv) * N * d) * (2 + 0.5 + 1 / 16)
     out = {
         "metric": "4-bit attn fwd TFLOPS (4*B*Hq*N^2*d, causal/2) and % of B200 dense FP4 peak",
@@ -262,7 +269,9 @@ def run_gpu(args):
         "quantize_qkv_gbs": round(quant_bytes / (k_quant * 1e-3) / 1e9, 1),
         "quantize_qkv_frac_hbm": round(quant_bytes / (k_quant * 1e-3) / 1e9 / hbm, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": None,
+                     "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                     "traffic": ATTN_TRAFFIC_BYTES if WORKLOAD == "qwen3-8b-4k" else None,
+                     "algorithmic_bytes": attn_bytes,
                      "peak_source": f"{src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)"},
         "e2e": {"value": round(e2e["tflops"], 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
