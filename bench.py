@@ -260,7 +260,7 @@ def run_gpu(args):
         "data": "synthetic (seeded Qwen3-8B-shaped post-RoPE Q/K/V, K outlier channels + bias)",
         "config": {"workload": WORKLOAD, "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
                    "kv_tile": w.bc, "smooth_qk_alpha": w.alpha,
-                   "l2": f"inputs rotated over {N_SETS} buffer sets (> 126 MB L2)", "parallelism": f"replicas x{world}"},
+                   "l2": l2_note(w), "parallelism": f"replicas x{world}"},
         "pct_fp4_peak": round(100 * agg["tflops"] / world / fp4_peak, 2),
         "pct_fp4_peak_datasheet_9pf": round(100 * agg["tflops"] / world / 9000.0, 2),
         "tokens_per_s": round(B * N * world / (agg["ms_per_step"] * 1e-3), 1),
@@ -370,6 +370,22 @@ def run_reference(args):
     print(json.dumps(out))
 
 
+def l2_note(w):
+    mb = N_SETS * 2 * w.B * (w.Hq + 2 * w.Hkv) * w.N * w.d / 1e6
+    rel = ">" if mb > 126 * 1.048576 else "<"
+    return f"inputs rotated over {N_SETS} buffer sets ({mb:.0f} MB of bf16 inputs {rel} 126 MB L2)"
+
+
+def set_workload(name):
+    global WORKLOAD, N_SETS
+    from bit_flashattention_b200 import configs
+    w = configs.get(name)
+    WORKLOAD = name
+    # rotate enough input sets that one step's bf16 inputs plus the rotation exceed 2x L2
+    set_bytes = 2 * w.B * (w.Hq + 2 * w.Hkv) * w.N * w.d
+    N_SETS = max(1, min(6, -(-(2 * 126 * 2 ** 20) // set_bytes)))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -378,7 +394,10 @@ def main(argv=None):
     ap.add_argument("--impl", default="hifa4", choices=["hifa4", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="one of tiny, qwen3-8b-4k (default), gemma2-9b-8k, llama3.1-8b-b4-16k, phi-32k")
     args = ap.parse_args(argv)
+    set_workload(args.workload)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
