@@ -274,6 +274,56 @@ OR_EXPORT void or_quantize_rows(const uint16_t* x, int B, int H, int Hkv, int N,
     }
 }
 
+/* Rotate-half RoPE in fp32 before Smooth-QK (the HiFA4 abstract applies the per-channel
+ * rescaling after RoPE), for the fused RoPE + Smooth-QK + quantise entry point.  Token n
+ * of every (b, h) sits at position n; its angle table is row n of cos, sin [N, d/2]
+ * (fp32, supplied by the caller).  With h = d/2, channel pair (i, i + h):
+ *   x'_i     = RN(RN(x_i * cos) - RN(x_{i+h} * sin))
+ *   x'_{i+h} = RN(RN(x_{i+h} * cos) + RN(x_i * sin)). */
+OR_EXPORT void or_rope_rows(const uint16_t* x, int B, int H, int N, int d, const float* cosv,
+                            const float* sinv, float* out) {
+    int half = d / 2;
+    long long rows = (long long)B * H * N;
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        int n = (int)(r % N);
+        const uint16_t* xr = x + r * d;
+        float* o = out + r * d;
+        for (int i = 0; i < half; ++i) {
+            float x1 = bf16_to_f32(xr[i]), x2 = bf16_to_f32(xr[i + half]);
+            float c = cosv[(long long)n * half + i], sn = sinv[(long long)n * half + i];
+            float a = x1 * c, b = x2 * sn;
+            o[i] = a - b;
+            float a2 = x2 * c, b2 = x1 * sn;
+            o[i + half] = a2 + b2;
+        }
+    }
+}
+
+/* or_quantize_rows on fp32 inputs (the rotated rows of or_rope_rows). */
+OR_EXPORT void or_quantize_rows_f32(const float* x, int B, int H, int Hkv, int N, int d,
+                                    const float* scale, uint8_t* codes, uint8_t* scales) {
+    int grp = H / Hkv;
+    long long rows = (long long)B * H * N;
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        int h = (int)((r / N) % H);
+        int g = h / grp;
+        const float* xr = x + r * d;
+        for (int blk = 0; blk < d / 16; ++blk) {
+            float v[16];
+            uint8_t c[16];
+            for (int i = 0; i < 16; ++i) {
+                float xv = xr[blk * 16 + i];
+                v[i] = scale ? xv * scale[g * d + blk * 16 + i] : xv;
+            }
+            quant16(v, c, &scales[r * (d / 16) + blk]);
+            for (int i = 0; i < 8; ++i)
+                codes[r * (d / 2) + blk * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+}
+
 /* V^T: v bf16 [B,Hkv,N,d] -> codes [B,Hkv,d,N/2], scales [B,Hkv,d,N/16]; blocks of 16
  * consecutive tokens of one channel, no smoothing. */
 OR_EXPORT void or_quantize_vt(const uint16_t* v, int B, int Hkv, int N, int d,
@@ -370,6 +420,10 @@ typedef struct {
     int state;        /* ST_MIRROR: fp16 m,l; fp32 O; alpha = E.  ST_F64: fp64 state, exact 2^x */
     int l_from_p;     /* 1: normaliser from unquantised P (the inconsistent formulation) */
     int s_model;
+    /* decode / split-KV (all 0 for the square forward): keys per kv head Nk (0 = N), the kv
+     * tile range [j0, j1) of this call, and dec_nq > 0 for packed decode rows: query row i
+     * holds token i % dec_nq, at position Nk - dec_nq + (i % dec_nq), which sees keys <= it */
+    int Nk, j0, j1, dec_nq;
 } loop_args;
 
 /* Per-row output and optional per-tile trace. */
@@ -381,12 +435,15 @@ typedef struct {
     float* tr_m;      /* m after tile j */
     float* tr_p;      /* [ntiles*bc] unquantised P of the tile (relative to that tile's m) */
     float* tr_phat;   /* [ntiles*bc] dequantised P_hat */
+    float* o_part;    /* [d] the unnormalised fp32 O accumulator at the end (mirror), may be NULL */
 } row_out;
 
 static void row_loop(const loop_args* a, long long row, row_out* out) {
     const int d = a->d, bc = a->bc, N = a->N;
+    const int Nk = a->Nk ? a->Nk : N;
     const long long bh = row / N;
     const int i = (int)(row % N);
+    const long long pos = a->dec_nq ? (long long)Nk - a->dec_nq + (i % a->dec_nq) : i;
     const int b = (int)(bh / a->Hq), h = (int)(bh % a->Hq);
     const int g = h / (a->Hq / a->Hkv);
     const long long kvh = (long long)b * a->Hkv + g;
@@ -394,6 +451,8 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
     const double cd = 1.4426950408889634074 / sqrt((double)d);
 
     int ntiles = a->causal ? i / bc + 1 : N / bc;
+    int jstart = 0;
+    if (a->dec_nq) { jstart = a->j0; ntiles = a->j1; }
     float m16 = -INFINITY, l16 = 0.0f;       /* mirror state */
     double m64 = -INFINITY, l64 = 0.0;       /* f64 state */
     float O32[256];
@@ -404,23 +463,23 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
     if (!a->quant)
         for (int x = 0; x < d; ++x) qd[x] = bf16_to_f32(a->q[row * d + x]);
 
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = jstart; j < ntiles; ++j) {
         double S[256];
         float Sf[256];
         int valid[256];
         double rowmax = -INFINITY;
         for (int kk = 0; kk < bc; ++kk) {
             int key = j * bc + kk;
-            valid[kk] = !(a->causal && key > i);
+            valid[kk] = a->dec_nq ? (key <= pos) : !(a->causal && key > i);
             if (!valid[kk]) { S[kk] = -INFINITY; Sf[kk] = -INFINITY; continue; }
             if (a->quant) {
                 Sf[kk] = s_dot(a->qc + row * (d / 2), a->qs + row * (d / 16),
-                               a->kc + (kvh * N + key) * (d / 2), a->ks + (kvh * N + key) * (d / 16),
+                               a->kc + (kvh * Nk + key) * (d / 2), a->ks + (kvh * Nk + key) * (d / 16),
                                d, a->s_model);
                 S[kk] = Sf[kk];
             } else {
                 double acc = 0.0;
-                for (int x = 0; x < d; ++x) acc += qd[x] * bf16_to_f32(a->k[(kvh * N + key) * d + x]);
+                for (int x = 0; x < d; ++x) acc += qd[x] * bf16_to_f32(a->k[(kvh * Nk + key) * d + x]);
                 S[kk] = acc;
                 Sf[kk] = (float)acc;
             }
@@ -442,8 +501,9 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
         }
         float mref = (a->state == ST_MIRROR || a->quant) ? mnew16 : (float)mnew64;
         if ((a->quant && mnew16 == -INFINITY) || (!a->quant && mnew64 == -INFINITY)) {
-            if (out->tr_m) out->tr_m[j] = mnew16;
-            if (out->tr_p) for (int kk = 0; kk < bc; ++kk) { out->tr_p[j * bc + kk] = 0; out->tr_phat[j * bc + kk] = 0; }
+            if (out->tr_m) out->tr_m[j - jstart] = mnew16;
+            if (out->tr_p)
+                for (int kk = 0; kk < bc; ++kk) { out->tr_p[(j - jstart) * bc + kk] = 0; out->tr_phat[(j - jstart) * bc + kk] = 0; }
             continue;                                         /* nothing seen yet: no-op tile */
         }
 
@@ -488,9 +548,9 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
                 double vv;
                 if (a->quant) {
                     long long vr = kvh * d + x;
-                    vv = (double)e2m1_value(nib(a->vc + vr * (N / 2), key)) * e4m3_value(a->vs[vr * (N / 16) + key / 16]);
+                    vv = (double)e2m1_value(nib(a->vc + vr * (Nk / 2), key)) * e4m3_value(a->vs[vr * (Nk / 16) + key / 16]);
                 } else {
-                    vv = bf16_to_f32(a->v[(kvh * N + key) * d + x]);
+                    vv = bf16_to_f32(a->v[(kvh * Nk + key) * d + x]);
                 }
                 pv[x] += Ph[kk] * vv;
             }
@@ -515,12 +575,17 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
             m16 = mnew16;
             m64 = mn;
         }
-        if (out->tr_m) out->tr_m[j] = a->quant ? mnew16 : (float)mnew64;
+        if (out->tr_m) out->tr_m[j - jstart] = a->quant ? mnew16 : (float)mnew64;
         if (out->tr_p)
-            for (int kk = 0; kk < bc; ++kk) { out->tr_p[j * bc + kk] = (float)P[kk]; out->tr_phat[j * bc + kk] = (float)Ph[kk]; }
+            for (int kk = 0; kk < bc; ++kk) {
+                out->tr_p[(j - jstart) * bc + kk] = (float)P[kk];
+                out->tr_phat[(j - jstart) * bc + kk] = (float)Ph[kk];
+            }
     }
 
     if (a->state == ST_MIRROR) {
+        if (out->o_part)
+            for (int x = 0; x < d; ++x) out->o_part[x] = O32[x];
         for (int x = 0; x < d; ++x) {
             float o = O32[x] / l16;
             if (out->o) out->o[x] = o;
@@ -592,6 +657,71 @@ OR_EXPORT int or_attn_trace(const uint8_t* qc, const uint8_t* qs, const uint8_t*
     row_loop(&a, row, &o);
     ml[0] = o.m;
     ml[1] = o.l;
+    return 0;
+}
+
+/* Decode / split-KV attention (a short query against a long key sequence).
+ * Q_hat is packed per (batch b, kv head g): [B, Hkv, 128, d] (plain code / scale layouts),
+ * row r = hi * nq + t holding token t of query head g * G + hi; rows >= G * nq are unused.
+ * Token t sits at position Nk - nq + t and sees the keys <= that position.  The Nk / bc kv
+ * tiles are cut into nsplit runs of T = ceil((Nk / bc) / nsplit) tiles; for every row and
+ * split s the tile loop of or_attn_fwd runs over the split's tiles from the initial state
+ * (m = -inf, l = 0, O = 0), giving m_s, l_s (fp16 values) and the fp32 accumulator O_s.
+ * The partials are merged in fp32, splits in order:
+ *   m = max_s m_s;  w_s = E(m_s - m) (0 when m_s = -inf, exactly 1 when m_s = m);
+ *   L = fma(w_s, l_s, L) from L = 0;  O = fma(w_s, O_s, O) from O = 0;
+ *   out = bf16_RN(RN(O * RN(1 / L))) (0 when L = 0);  m_out = m, l_out = fp16_RN(L).
+ * o_bf16: [B, Hkv * G, nq, d]; m_out, l_out: [B, Hkv * G, nq] (fp32 holding the values);
+ * part_o [B * Hkv, nsplit, 128, d] and part_ml [B * Hkv, nsplit, 128, 2] (may be NULL)
+ * receive the partials of the used rows. */
+OR_EXPORT int or_attn_decode(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
+                             const uint8_t* vtc, const uint8_t* vts, int B, int Hkv, int G, int nq, int Nk, int d,
+                             int bc, int nsplit, int s_model, uint16_t* o_bf16, float* m_out, float* l_out,
+                             float* part_o, float* part_ml) {
+    if (d % 16 || d > 256 || bc % 16 || bc > 256 || Nk % bc || G * nq > 128 || nsplit < 1 || nsplit > 64) return -1;
+    const int ntile = Nk / bc, T = (ntile + nsplit - 1) / nsplit;
+    const long long nrows = (long long)B * Hkv * G * nq;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long long idx = 0; idx < nrows; ++idx) {
+        const long long bkv = idx / (G * nq);
+        const int r = (int)(idx % (G * nq));
+        float mp[64], lp[64];
+        static __thread float op[64][256];
+        for (int sp = 0; sp < nsplit; ++sp) {
+            int j0 = sp * T, j1 = j0 + T < ntile ? j0 + T : ntile;
+            if (j0 > ntile) j0 = ntile;
+            /* the packed rows form Hkv "heads" of 128 query rows each */
+            loop_args a = {qc, qs, kc, ks, vtc, vts, NULL, NULL, NULL, B, Hkv, Hkv, 128, d, 0, bc,
+                           1, ST_MIRROR, 0, s_model, Nk, j0, j1, nq};
+            double o64[256];
+            row_out o = {o64, NULL, 0, 0, NULL, NULL, NULL, op[sp]};
+            row_loop(&a, bkv * 128 + r, &o);
+            if (j0 >= j1) { o.m = -INFINITY; o.l = 0.0f; for (int x = 0; x < d; ++x) op[sp][x] = 0.0f; }
+            mp[sp] = o.m;
+            lp[sp] = o.l;
+            if (part_o)
+                for (int x = 0; x < d; ++x) part_o[((bkv * nsplit + sp) * 128 + r) * d + x] = op[sp][x];
+            if (part_ml) {
+                part_ml[((bkv * nsplit + sp) * 128 + r) * 2] = o.m;
+                part_ml[((bkv * nsplit + sp) * 128 + r) * 2 + 1] = o.l;
+            }
+        }
+        float m = -INFINITY;
+        for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, mp[sp]);
+        float L = 0.0f, O[256];
+        for (int x = 0; x < d; ++x) O[x] = 0.0f;
+        for (int sp = 0; sp < nsplit; ++sp) {
+            float w = (mp[sp] == -INFINITY) ? 0.0f : own_exp2(mp[sp] - m);
+            L = fmaf(w, lp[sp], L);
+            for (int x = 0; x < d; ++x) O[x] = fmaf(w, op[sp][x], O[x]);
+        }
+        const int hi = r / nq, t = r % nq;
+        const long long orow = ((bkv / Hkv) * (long long)(Hkv * G) + (bkv % Hkv) * G + hi) * nq + t;
+        float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+        for (int x = 0; x < d; ++x) o_bf16[orow * d + x] = f32_to_bf16(O[x] * inv);
+        m_out[orow] = m;
+        l_out[orow] = f16_round(L);
+    }
     return 0;
 }
 

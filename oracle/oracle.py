@@ -54,6 +54,10 @@ def lib():
         L.or_calibrate.argtypes = [P, P, i, i, i, i, i, dbl, P, P]
         L.or_quantize_rows.argtypes = [P, i, i, i, i, i, P, P, P]
         L.or_quantize_vt.argtypes = [P, i, i, i, i, P, P]
+        L.or_rope_rows.argtypes = [P, i, i, i, i, P, P, P]
+        L.or_attn_decode.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, P, P, P, P, P]
+        L.or_attn_decode.restype = i
+        L.or_quantize_rows_f32.argtypes = [P, i, i, i, i, i, P, P, P]
         L.or_qk_scores.argtypes = [P, P, P, P, i, i, i, i, P]
         L.or_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, P, ll, P, P, P, P]
         L.or_attn_fwd.restype = i
@@ -164,6 +168,35 @@ def quantize_rows(x, Hkv, scale=None):
     return codes, scales
 
 
+def rope_rows(x, cos, sin):
+    """Rotate-half RoPE of bf16 bits [B,H,N,d] with fp32 angle tables cos, sin [N, d/2]
+    (row n = position of token n), in fp32 with each product and sum rounded once."""
+    x = _c(x, np.uint16)
+    B, H, N, d = x.shape
+    cos = _c(cos, np.float32)
+    sin = _c(sin, np.float32)
+    assert cos.shape == (N, d // 2) and sin.shape == (N, d // 2)
+    out = np.empty((B, H, N, d), np.float32)
+    lib().or_rope_rows(_p(x), B, H, N, d, _p(cos), _p(sin), _p(out))
+    return out
+
+
+def quantize_rows_f32(x, Hkv, scale=None):
+    """quantize_rows on fp32 inputs [B,H,N,d]."""
+    x = _c(x, np.float32)
+    B, H, N, d = x.shape
+    codes = np.empty((B, H, N, d // 2), np.uint8)
+    scales = np.empty((B, H, N, d // 16), np.uint8)
+    sc = None if scale is None else _c(scale, np.float32)
+    lib().or_quantize_rows_f32(_p(x), B, H, Hkv, N, d, _p(sc), _p(codes), _p(scales))
+    return codes, scales
+
+
+def quantize_rows_rope(x_pre, Hkv, cos, sin, scale=None):
+    """The fused entry point: RoPE (rope_rows), then Smooth-QK and the 4-bit quantiser."""
+    return quantize_rows_f32(rope_rows(x_pre, cos, sin), Hkv, scale)
+
+
 def quantize_vt(v):
     v = _c(v, np.uint16)
     B, Hkv, N, d = v.shape
@@ -223,6 +256,39 @@ def attn_fwd(qz: Quantized, causal, bc, rows=None, state=STATE_MIRROR, l_from_p=
     if want_f64:
         out["o_f64"] = o64
     return out
+
+
+def pack_decode_q(q, Hkv):
+    """Decode rows of bf16 bits Q [B, Hq, nq, d] packed per kv head: [B, Hkv, 128, d], row
+    r = hi * nq + t = token t of query head g * G + hi (G = Hq / Hkv); rows >= G * nq zero."""
+    q = _c(q, np.uint16)
+    B, Hq, nq, d = q.shape
+    G = Hq // Hkv
+    assert G * nq <= 128
+    out = np.zeros((B, Hkv, 128, d), np.uint16)
+    out[:, :, : G * nq] = q.reshape(B, Hkv, G * nq, d)
+    return out
+
+
+def attn_decode(qc, qs, kc, ks, vc, vs, G, nq, bc, nsplit, s_model=S_MODEL_DEFAULT):
+    """Decode / split-KV attention on the packed Q_hat (codes [B, Hkv, 128, d/2], scales
+    [B, Hkv, 128, d/16]) and K_hat, V_hat^T of Nk keys; see or_attn_decode.  Returns
+    dict o_bf16 [B, Hkv*G, nq, d] (uint16), m, l [B, Hkv*G, nq], part_o, part_ml."""
+    qc, qs, kc, ks, vc, vs = (_c(a, np.uint8) for a in (qc, qs, kc, ks, vc, vs))
+    B, Hkv, R, half = qc.shape
+    d = 2 * half
+    Nk = kc.shape[2]
+    assert R == 128
+    o = np.empty((B, Hkv * G, nq, d), np.uint16)
+    m = np.empty((B, Hkv * G, nq), np.float32)
+    l = np.empty((B, Hkv * G, nq), np.float32)
+    po = np.zeros((B * Hkv, nsplit, 128, d), np.float32)
+    pml = np.zeros((B * Hkv, nsplit, 128, 2), np.float32)
+    rc = lib().or_attn_decode(_p(qc), _p(qs), _p(kc), _p(ks), _p(vc), _p(vs), B, Hkv, G, nq, Nk, d, bc, nsplit,
+                              s_model, _p(o), _p(m), _p(l), _p(po), _p(pml))
+    if rc != 0:
+        raise ValueError("oracle rejected the decode shape")
+    return {"o_bf16": o, "m": m, "l": l, "part_o": po, "part_ml": pml}
 
 
 def attn_trace(qz: Quantized, causal, bc, row, state=STATE_MIRROR, l_from_p=False, s_model=S_MODEL_DEFAULT):
