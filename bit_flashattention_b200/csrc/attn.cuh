@@ -59,7 +59,8 @@ struct AttnCfg {
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
   static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 128 x fp32 table of L(sigma)
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
-  static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 128 * 4;
+  static constexpr uint32_t OFF_XSUM = OFF_XMAX + 2 * 4 * 128 * 4;   // [2][NSW][128] partial sums of P (ablation)
+  static constexpr uint32_t OFF_BAR = OFF_XSUM + 2 * 4 * 128 * 4;
   // barriers: q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
   // s_full[2], s_empty[2], p_full[2], o_bar, o_free, drain[2]
   static constexpr int NBAR = 4 + 2 * KS + 2 * VS + 6 + 4;
@@ -100,6 +101,16 @@ struct AttnParams {
   float c;                  // RN(log2(e) / sqrt(D))
   unsigned long long wait_ns;
   int inject;               // 1: the producer never delivers kv tile 1 (timeout test)
+  int l_from_p;             // ablation kernels: 1 = l from the unquantised P (inconsistent normaliser)
+  // keys per kv head (= N for the square forward); decode / split-KV kernels (DEC): Q holds
+  // packed rows (B * Hkv tiles of 128 rows: row r = hi * nq + t, token t of query head
+  // g * G + hi, at position Nk - nq + t); unit = (b * Hkv + g, split) over kv tiles
+  // [split * tps, ...); partials (unnormalised fp32 O, m, l) go to part_*
+  int Nk, nq, G, nsplit, tps;
+  float* part_o;            // [B * Hkv * nsplit * 128, D]
+  float* part_m;            // [B * Hkv * nsplit * 128]
+  float* part_l;
+  float* trace;             // ablation kernels: [B*Hq*N][N/BC][2] per (row, tile): sum P_hat, sum P; or nullptr
   float lneg[128];          // L(sigma) = RN(-log2 sigma) per E4M3 scale code (-inf for 0)
 };
 
@@ -133,23 +144,45 @@ __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Work unit u (0 <= u < B*Hq*(N/128)) -> (batch*head, query tile); causal units are
-// ordered longest first (the last query tiles need the most kv tiles).
-__device__ __forceinline__ void unit_coords(int u, const AttnParams& p, int& bh, int& qtile) {
-  const int BH = p.B * p.Hq, nqt = p.N / 128;
-  qtile = p.causal ? nqt - 1 - u / BH : u / BH;
-  bh = u % BH;
+// Geometry of work unit u.  Square forward: units (batch * query head, 128-row query tile),
+// causal ones longest first; decode: units (batch * kv head, split).
+struct UnitGeom {
+  int qrow;         // first row of the unit's Q tile in the Q tensor (its scale atom: qrow / 128)
+  int kvh;          // global kv head b * Hkv + g
+  int j0, nt;       // kv tiles j0 .. j0 + nt - 1
+  long long orow;   // output row of TMEM lane 0 (decode: partial slot u * 128)
+  int pos0;         // square causal: the key limit of lane 0 (lane r sees keys <= pos0 + r)
+};
+
+template <int BC, bool DEC>
+__device__ __forceinline__ UnitGeom unit_geom(int u, const AttnParams& p) {
+  UnitGeom g;
+  if constexpr (DEC) {
+    const int bkv = u / p.nsplit, sp = u % p.nsplit, ntile = p.Nk / BC;
+    g.qrow = bkv * 128;
+    g.kvh = bkv;
+    g.j0 = min(sp * p.tps, ntile);
+    g.nt = min(p.tps, ntile - g.j0);
+    g.orow = (long long)u * 128;
+    g.pos0 = 0;
+  } else {
+    const int BH = p.B * p.Hq, nqt = p.N / 128;
+    const int qtile = p.causal ? nqt - 1 - u / BH : u / BH;
+    const int bh = u % BH;
+    g.qrow = bh * p.N + qtile * 128;
+    g.kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
+    g.j0 = 0;
+    g.nt = p.causal ? ((qtile + 1) * 128 + BC - 1) / BC : p.N / BC;
+    g.orow = (long long)bh * p.N + qtile * 128;
+    g.pos0 = qtile * 128;
+  }
+  return g;
 }
 
-template <int BC>
-__device__ __forceinline__ int unit_tiles(int qtile, const AttnParams& p) {
-  return p.causal ? ((qtile + 1) * 128 + BC - 1) / BC : p.N / BC;
-}
-
-// Persistent kernel: each CTA walks its share of the units (see unit_of).  Ring-buffer
-// phases run on a tile counter g that continues across units; the Q tile is
-// double-buffered so the next unit's Q arrives while the current one is processed.
-template <int D, int BC>
+//
+// DEC: the decode / split-KV kernels (packed query rows, a split's tile range, partial
+// outputs); the square forward is the DEC = false instance.
+template <int D, int BC, bool SUMP = false, bool DEC = false>
 __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
@@ -183,8 +216,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   auto sPsf = [&](int s) { return smem + C::OFF_PSF + s * C::SZ_PSF; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nqt = p.N / 128;
-  const int units = p.B * p.Hq * nqt;
+  const int units = DEC ? p.B * p.Hkv * p.nsplit : p.B * p.Hq * (p.N / 128);
   // the CTA's i-th unit: rows of gridDim.x units, every other row reversed (snake order),
   // which evens out the per-CTA work of the longest-first causal list
   auto unit_of = [&](int i) {
@@ -202,6 +234,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
   }
   float* rtab = reinterpret_cast<float*>(smem + C::OFF_RTAB);
   float* xmax = reinterpret_cast<float*>(smem + C::OFF_XMAX);
+  float* xsum = reinterpret_cast<float*>(smem + C::OFF_XSUM);
   if (warp >= 3) {
     // the ones operand (E2M1 1.0 = 0b0010 in both nibbles) and its scales (UE4M3 1.0)
     const int t = threadIdx.x - 96, nt2 = 128 * C::NSW;
@@ -228,28 +261,28 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       int nq = 0, nk = 0, nv = 0;   // loads issued (Q per unit, K and V per tile)
       bool ok = true;
       for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
-        int bh, qtile;
-        unit_coords(u, p, bh, qtile);
-        const int kvh = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
-        const int nt = unit_tiles<BC>(qtile, p);
+        const UnitGeom ug = unit_geom<BC, DEC>(u, p);
+        const int kvh = ug.kvh;
         const int qb = i & 1;
         if (i >= 2 && !mbar_wait(&q_empty[qb], ((i >> 1) - 1) & 1, abort, p.status, p.wait_ns)) break;
         mbar_arrive_expect_tx(&q_full[qb], C::SZ_Q + C::SZ_QSF);
-        tma_load_2d(sQ(qb), &tmQ, 0, bh * p.N + qtile * 128, &q_full[qb]);
-        bulk_load(sQsf(qb), p.qsf + ((long long)bh * nqt + qtile) * C::SZ_QSF, C::SZ_QSF, &q_full[qb]);
+        tma_load_2d(sQ(qb), &tmQ, 0, ug.qrow, &q_full[qb]);
+        bulk_load(sQsf(qb), p.qsf + (long long)(ug.qrow / 128) * C::SZ_QSF, C::SZ_QSF, &q_full[qb]);
         ++nq;
-        for (int j = 0; j < nt; ++j) {
-          if (p.inject == 1 && i == 0 && j == 1) { ok = false; break; }
+        for (int jj = 0; jj < ug.nt; ++jj) {
+          const int j = ug.j0 + jj;
+          if (p.inject == 1 && i == 0 && jj == 1) { ok = false; break; }
           const int g = nk, ks = g % C::KS, vs = g % C::VS;
           if (g >= C::KS && !mbar_wait(&k_empty[ks], ((g / C::KS) - 1) & 1, abort, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&k_full[ks], C::SZ_K + C::SZ_KSF);
-          tma_load_2d(sK(ks), &tmK, 0, kvh * p.N + j * BC, &k_full[ks]);
+          tma_load_2d(sK(ks), &tmK, 0, kvh * p.Nk + j * BC, &k_full[ks]);
           // the tile's NAK consecutive 128-row atoms (KQ x 512 bytes each) are contiguous
           const int katom = (j * BC) / 128;
-          bulk_load(sKsf(ks), p.ksf + ((long long)kvh * nqt + katom) * (C::KQ * 512), C::SZ_KSF, &k_full[ks]);
+          bulk_load(sKsf(ks), p.ksf + ((long long)kvh * (p.Nk / 128) + katom) * (C::KQ * 512), C::SZ_KSF,
+                    &k_full[ks]);
           ++nk;
           if (g >= C::VS && !mbar_wait(&v_empty[vs], ((g / C::VS) - 1) & 1, abort, p.status, p.wait_ns)) {
             ok = false;
@@ -257,7 +290,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           }
           mbar_arrive_expect_tx(&v_full[vs], C::SZ_V + C::SZ_VSF);
           tma_load_2d(sV(vs), &tmV, j * C::PROW, kvh * D, &v_full[vs]);
-          bulk_load(sVsf(vs), p.vsf + ((long long)kvh * (p.N / 64) + j * C::KP) * (C::NAV * 512), C::SZ_VSF,
+          bulk_load(sVsf(vs), p.vsf + ((long long)kvh * (p.Nk / 64) + j * C::KP) * (C::NAV * 512), C::SZ_VSF,
                     &v_full[vs]);
           ++nv;
         }
@@ -286,9 +319,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     bool ok = true;
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
-      int bh, qtile;
-      unit_coords(u, p, bh, qtile);
-      const int nt = unit_tiles<BC>(qtile, p);
+      const UnitGeom ug = unit_geom<BC, DEC>(u, p);
+      const int nt = ug.nt;
       const int qb = i & 1;
       ok = wait_all(&q_full[qb], (i >> 1) & 1, abort, p.status, p.wait_ns);
       // the previous unit's QK MMAs (which read the Q scale columns) have completed
@@ -302,7 +334,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       }
       __syncwarp();
       const uint64_t dQi = dQ + ((qb * align_up(C::SZ_Q, 1024)) >> 4);
-      for (int j = 0; ok && j < nt; ++j, ++g) {
+      for (int jj = 0; ok && jj < nt; ++jj, ++g) {
+        const int j = ug.j0 + jj;
         const int ks = g % C::KS, sb = g % C::SB;
         ok = wait_all(&k_full[ks], (g / C::KS) & 1, abort, p.status, p.wait_ns);
         if (ok && g >= C::SB) ok = wait_all(&s_empty[sb], ((g / C::SB) - 1) & 1, abort, p.status, p.wait_ns);
@@ -335,7 +368,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
                      sfk + 4 * C::NAK * kc, kc > 0 ? 1u : 0u);
           tc_commit(&s_full[sb]);
           tc_commit(&k_empty[ks]);
-          if (j == nt - 1) tc_commit(&q_empty[qb]);   // the unit's Q tile and Q scales are free
+          if (jj == nt - 1) tc_commit(&q_empty[qb]);   // the unit's Q tile and Q scales are free
         }
         __syncwarp();
       }
@@ -362,10 +395,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     bool ok = true;
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
-      int bh, qtile;
-      unit_coords(u, p, bh, qtile);
-      const int nt = unit_tiles<BC>(qtile, p);
-      for (int j = 0; ok && j < nt; ++j, ++g) {
+      const int nt = unit_geom<BC, DEC>(u, p).nt;
+      for (int j = 0; ok && j < nt; ++j, ++g) {   // j: the unit's local tile index
         const int vs = g % C::VS, pb = g & 1;
         ok = wait_all(&v_full[vs], (g / C::VS) & 1, abort, p.status, p.wait_ns);
         ok = ok && wait_all(&p_full[pb], (g >> 1) & 1, abort, p.status, p.wait_ns);
@@ -415,15 +446,47 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     const float c = p.c;
     const float c7 = c * 0.0078125f;
     // Epilogue of a unit whose last tile is gl: read R and O of that tile's PV, release
-    // them (o_free), then O / l -> bf16.  It runs after the next unit's first tile, which
-    // touches neither O nor R, so that tile's work overlaps the last PV.
-    auto epilogue = [&](int gl, long long orow, float l_e, float alpha_e) -> bool {
+    // them (o_free), then O / l -> bf16 (decode: the unnormalised fp32 O and l of the
+    // split's partial).  It runs after the next unit's first tile, which touches neither O
+    // nor R, so that tile's work overlaps the last PV.
+    const int ntmax = p.N / BC;
+    auto epilogue = [&](int gl, long long orow, float l_e, float alpha_e, float rsum_e, int jl) -> bool {
       if (!wait_all(o_bar, gl & 1, abort, p.status, p.wait_ns)) return false;
       tc_fence_after();
       uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
       tmem_wait_ld();
       reg_fence(rr);
-      const float l_fin = f16_round(__fmaf_rn(alpha_e, l_e, __uint_as_float(rr[0])));
+      float r_use = __uint_as_float(rr[0]);
+      if constexpr (SUMP) {
+        if (p.trace && wg == 0) {
+          float* t = p.trace + (orow * ntmax + jl) * 2;
+          t[0] = r_use;
+          t[1] = rsum_e;
+        }
+        if (p.l_from_p) r_use = rsum_e;
+      }
+      const float l_fin = f16_round(__fmaf_rn(alpha_e, l_e, r_use));
+      if constexpr (DEC) {
+        float4* pdst = reinterpret_cast<float4*>(p.part_o + orow * D);
+#pragma unroll 1
+        for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tbase + lrow + C::T_O + c0, o);
+          tmem_wait_ld();
+          reg_fence(o);
+          if (c0 + 32 == wg * OW + OW) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            pdst[c0 / 4 + q] = make_float4(__uint_as_float(o[4 * q]), __uint_as_float(o[4 * q + 1]),
+                                           __uint_as_float(o[4 * q + 2]), __uint_as_float(o[4 * q + 3]));
+        }
+        if (wg == 0) p.part_l[orow] = l_fin;
+        return true;
+      }
       const float inv = (l_fin > 0.0f) ? __frcp_rn(l_fin) : 0.0f;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
 #pragma unroll 1
@@ -454,14 +517,26 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     bool ok = true;
     long long pend_row = 0;                  // the previous unit's output row, l and alpha
     float pend_l = 0.0f, pend_alpha = 0.0f;
+    float pend_rsum = 0.0f;                  // ablation kernels: its last tile's sum of P and index
+    int pend_j = 0;
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
-      int bh, qtile;
-      unit_coords(u, p, bh, qtile);
-      const int nt = unit_tiles<BC>(qtile, p);
-      const int qrow = qtile * 128 + row;
+      const UnitGeom ug = unit_geom<BC, DEC>(u, p);
+      const int nt = ug.nt;
+      // the last key this thread's row sees, and the smallest such limit of the unit's rows:
+      // tiles ending at or below it need no mask
+      int pos, pos_min;
+      if constexpr (DEC) {
+        pos = row < p.G * p.nq ? p.Nk - p.nq + row % p.nq : p.Nk - 1;
+        pos_min = p.Nk - p.nq;
+      } else {
+        pos = p.causal ? ug.pos0 + row : 0x7FFFFFFF;
+        pos_min = p.causal ? ug.pos0 : 0x7FFFFFFF;
+      }
       float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
-      for (int j = 0; j < nt; ++j, ++g) {
+      float rsum_prev = 0.0f;                // ablation kernels: the previous tile's sum of P
+      for (int jj = 0; jj < nt; ++jj, ++g) {
+        const int j = ug.j0 + jj;
         const int sb = g % C::SB, pb = g & 1;
         ok = wait_all(&s_full[sb], (g / C::SB) & 1, abort, p.status, p.wait_ns);
         if (!ok) break;
@@ -480,10 +555,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[sb]);
-        if (p.causal && (j + 1) * BC - 1 > qtile * 128) {
+        if ((j + 1) * BC - 1 > pos_min) {
 #pragma unroll
           for (int q = 0; q < CW; ++q)
-            if (j * BC + col0 + q > qrow) s[q] = -INFINITY;
+            if (j * BC + col0 + q > pos) s[q] = -INFINITY;
         }
         float bmax[NB];
 #pragma unroll
@@ -510,6 +585,21 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
             (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
         const float negm = -mnew;
         const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
+        float rsum = 0.0f;
+        if constexpr (SUMP) {
+          float part = 0.0f;
+#pragma unroll
+          for (int e = 0; e < CW; e += 2) {
+            const float2 e2 = exp2_own2(__ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2));
+            part = __fadd_rn(__fadd_rn(part, e2.x), e2.y);
+          }
+          float* xs = xsum + (g & 1) * (C::NSW * 128);
+          xs[wg * 128 + row] = part;
+          named_bar(1 + q4, 32 * C::NSW);
+          rsum = xs[row];
+#pragma unroll
+          for (int w2 = 1; w2 < C::NSW; ++w2) rsum = __fadd_rn(rsum, xs[w2 * 128 + row]);
+        }
         // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call
         float pmax[NB];
 #pragma unroll
@@ -548,14 +638,23 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
         }
         fence_proxy_async_smem();
-        if (j > 0) {
+        if (jj > 0) {
           ok = wait_all(o_bar, (g - 1) & 1, abort, p.status, p.wait_ns);
           if (!ok) break;
           tc_fence_after();
           uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
           tmem_wait_ld();
           reg_fence(rr);
-          l_run = f16_round(__fmaf_rn(alpha_prev, l_run, __uint_as_float(rr[0])));
+          float r_use = __uint_as_float(rr[0]);
+          if constexpr (SUMP) {
+            if (p.trace && wg == 0) {
+              float* t = p.trace + ((ug.orow + row) * ntmax + (j - 1)) * 2;
+              t[0] = r_use;
+              t[1] = rsum_prev;
+            }
+            if (p.l_from_p) r_use = rsum_prev;
+          }
+          l_run = f16_round(__fmaf_rn(alpha_prev, l_run, r_use));
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
             for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
@@ -580,24 +679,69 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         if (lane == 0) mbar_arrive(&p_full[pb]);
         alpha_prev = alpha;
         m_run = mnew;
-        if (j == 0 && i > 0) {
-          ok = epilogue(g - 1, pend_row, pend_l, pend_alpha);
+        rsum_prev = rsum;
+        if (jj == 0 && i > 0) {
+          ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j);
           if (!ok) break;
         }
       }
       if (!ok) break;
-      pend_row = (long long)bh * p.N + qrow;
+      pend_row = ug.orow + row;
       pend_l = l_run;
       pend_alpha = alpha_prev;
-      if (wg == 0 && p.m_out) p.m_out[pend_row] = __float2half_rn(m_run);
+      pend_rsum = rsum_prev;
+      pend_j = ug.j0 + nt - 1;
+      if (wg == 0) {
+        if constexpr (DEC) p.part_m[pend_row] = m_run;
+        else if (p.m_out) p.m_out[pend_row] = __float2half_rn(m_run);
+      }
     }
-    if (ok && g > 0) ok = epilogue(g - 1, pend_row, pend_l, pend_alpha);
+    if (ok && g > 0) ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- decode merge
+// Merge of the split partials of one packed decode row per CTA (thread x = output channel
+// x): m = max_s m_s, w_s = E(m_s - m) (0 when m_s = -inf), L = fma(w_s, l_s, L) and
+// O = fma(w_s, O_s, O) over the splits in order, out = bf16(O * RN(1/L)), m and fp16(L)
+// out.  o: [B, Hq, nq, D]; rows r = hi * nq + t of kv head g are token t of head g * G + hi.
+struct DecodeMergeArgs {
+  const float* part_o;
+  const float* part_m;
+  const float* part_l;
+  __nv_bfloat16* o;
+  __half* m_out;
+  __half* l_out;
+  int Hkv, G, nq, nsplit;
+};
+
+template <int D>
+__global__ void __launch_bounds__(D) k_decode_merge(const DecodeMergeArgs a) {
+  const int rows = a.G * a.nq;
+  const int bkv = blockIdx.x / rows, r = blockIdx.x % rows, x = threadIdx.x;
+  float m = -INFINITY;
+  for (int s = 0; s < a.nsplit; ++s) m = fmaxf(m, a.part_m[((long long)bkv * a.nsplit + s) * 128 + r]);
+  float L = 0.0f, O = 0.0f;
+  for (int s = 0; s < a.nsplit; ++s) {
+    const long long slot = ((long long)bkv * a.nsplit + s) * 128 + r;
+    const float ms = a.part_m[slot];
+    const float w = (ms == -INFINITY) ? 0.0f : exp2_own(__fsub_rn(ms, m));
+    L = __fmaf_rn(w, a.part_l[slot], L);
+    O = __fmaf_rn(w, a.part_o[slot * D + x], O);
+  }
+  const float inv = (L > 0.0f) ? __frcp_rn(L) : 0.0f;
+  const int b = bkv / a.Hkv, g = bkv % a.Hkv, hi = r / a.nq, t = r % a.nq;
+  const long long orow = ((long long)b * a.Hkv * a.G + g * a.G + hi) * a.nq + t;
+  a.o[orow * D + x] = __float2bfloat16_rn(__fmul_rn(O, inv));
+  if (x == 0) {
+    if (a.m_out) a.m_out[orow] = __float2half_rn(m);
+    if (a.l_out) a.l_out[orow] = __float2half_rn(L);
   }
 }
 

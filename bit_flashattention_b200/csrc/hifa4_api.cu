@@ -135,19 +135,28 @@ void fill_neg_log2_scales(float* t) {
   }
 }
 
-template <int D, int BC>
+// Decode / split-KV launch parameters (see AttnParams).
+struct DecodeSpec {
+  int nq, G, Nk, nsplit, tps;
+  float *part_o, *part_m, *part_l;
+};
+
+template <int D, int BC, bool SUMP = false, bool DEC = false>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
-                int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
+                int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream,
+                int l_from_p = 0, float* trace = nullptr, const DecodeSpec* dec = nullptr) {
   using C = AttnCfg<D, BC>;
+  const int Nk = dec ? dec->Nk : N;
+  const uint64_t qrows = dec ? (uint64_t)B * Hkv * 128 : (uint64_t)B * Hq * N;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q->codes, D / 2, (uint64_t)B * Hq * N, D / 2, D / 2, 128) ||
-      !make_map(&tk, k->codes, D / 2, (uint64_t)B * Hkv * N, D / 2, D / 2, BC) ||
-      !make_map(&tv, vt->codes, N / 2, (uint64_t)B * Hkv * D, N / 2, BC / 2, D))
+  if (!make_map(&tq, q->codes, D / 2, qrows, D / 2, D / 2, 128) ||
+      !make_map(&tk, k->codes, D / 2, (uint64_t)B * Hkv * Nk, D / 2, D / 2, BC) ||
+      !make_map(&tv, vt->codes, Nk / 2, (uint64_t)B * Hkv * D, Nk / 2, BC / 2, D))
     return HIFA4_ERR_CUDA;
   // One CTA per SM when it holds all 512 TMEM columns: ask for more than half the SM's
   // shared memory so a second CTA cannot become resident and block in tcgen05.alloc.
   const uint32_t smem = (C::TMEM_COLS == 512 && C::SMEM < 120 * 1024) ? 120 * 1024 : C::SMEM;
-  static bool attr = set_smem(k_attn_fwd<D, BC>, smem);
+  static bool attr = set_smem(k_attn_fwd<D, BC, SUMP, DEC>, smem);
   if (!attr) return HIFA4_ERR_CUDA;
   AttnParams p;
   p.qsf = static_cast<const uint8_t*>(q->scales);
@@ -165,20 +174,63 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   p.c = (float)(1.4426950408889634074 / std::sqrt((double)D));
   p.wait_ns = g_wait_ns;
   p.inject = g_inject;
+  p.l_from_p = l_from_p;
+  p.trace = trace;
+  p.Nk = Nk;
+  p.nq = dec ? dec->nq : 1;
+  p.G = dec ? dec->G : 1;
+  p.nsplit = dec ? dec->nsplit : 1;
+  p.tps = dec ? dec->tps : 0;
+  p.part_o = dec ? dec->part_o : nullptr;
+  p.part_m = dec ? dec->part_m : nullptr;
+  p.part_l = dec ? dec->part_l : nullptr;
+  if (dec) {
+    p.N = 128;
+    p.causal = 0;
+  }
   fill_neg_log2_scales(p.lneg);
   // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM)
   static int per_sm = 0;
   if (per_sm == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC>, C::NTHREADS, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem) != cudaSuccess ||
         n <= 0)
       n = 1;
     per_sm = n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
   }
-  const long long units = (long long)B * Hq * (N / 128), cap = (long long)per_sm * num_sms();
+  const long long units = dec ? (long long)B * Hkv * dec->nsplit : (long long)B * Hq * (N / 128);
+  const long long cap = (long long)per_sm * num_sms();
   const unsigned grid = (unsigned)(units < cap ? units : cap);
-  k_attn_fwd<D, BC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
+  k_attn_fwd<D, BC, SUMP, DEC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
+}
+
+// Validation and dispatch shared by the plain and the ablation entry points.
+template <bool SUMP>
+int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
+                  int N, int d, int causal, int kv_tile, void* o, void* m_out, void* l_out, int* status,
+                  cudaStream_t stream, int l_from_p, float* trace) {
+  if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
+    return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : (d == 128 ? 256 : 128);
+  if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (d == 64 && kv_tile == 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (N % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q, B, Hq, N, d, 0) || !qt_ok(k, B, Hkv, N, d, 0) || !qt_ok(vt, B, Hkv, N, d, 1))
+    return HIFA4_ERR_INVALID_ARG;
+  if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+#define HIFA4_LAUNCH(DD, BB) \
+  launch_attn<DD, BB, SUMP>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, l_from_p, trace)
+  if (d == 64) return kv_tile == 64 ? HIFA4_LAUNCH(64, 64) : HIFA4_LAUNCH(64, 128);
+  if (d == 128) {
+    if (kv_tile == 256) return HIFA4_LAUNCH(128, 256);
+    return kv_tile == 64 ? HIFA4_LAUNCH(128, 64) : HIFA4_LAUNCH(128, 128);
+  }
+  return HIFA4_LAUNCH(256, 64);
+#undef HIFA4_LAUNCH
 }
 
 }  // namespace
@@ -261,8 +313,10 @@ int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], 
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   const int rows = d == 256 ? 64 : 128;   // rows per unit of k_quant_rows<d>
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
+                   nullptr, nullptr, 0, 0,
                    static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
+                   nullptr, nullptr, 0, 0,
                    static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
   const int units = qa.units + ka.units;
   switch (d) {
@@ -271,6 +325,47 @@ int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], 
     default: k_quant_rows<256><<<resident_grid(k_quant_rows<256>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
   }
   return cuda_status(cudaGetLastError());
+}
+
+int hifa4_quantize_qk_rope(const void* q, const void* k, const int64_t q_strides[3], const int64_t k_strides[3],
+                           int B, int Hq, int Hkv, int N, int d, const float* rope_cos, const float* rope_sin,
+                           const float* s, const float* sinv, const hifa4_qtensor* q_out, const hifa4_qtensor* k_out,
+                           int* status, cudaStream_t stream) {
+  if (!strides_ok(q, q_strides) || !strides_ok(k, k_strides) || !status || ((s == nullptr) != (sinv == nullptr)) ||
+      (s && (!aligned16(s) || !aligned16(sinv))) || !rope_cos || !rope_sin || !aligned16(rope_cos) ||
+      !aligned16(rope_sin))
+    return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0)) return HIFA4_ERR_INVALID_ARG;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  const int rows = d == 256 ? 64 : 128;
+  QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
+                   rope_cos, rope_sin, 0, 0, static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales),
+                   B * Hq * (N / rows)};
+  QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
+                   rope_cos, rope_sin, 0, 0, static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales),
+                   B * Hkv * (N / rows)};
+  const int units = qa.units + ka.units;
+  switch (d) {
+    case 64: k_quant_rows_rope<64><<<resident_grid(k_quant_rows_rope<64>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
+    case 128: k_quant_rows_rope<128><<<resident_grid(k_quant_rows_rope<128>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
+    default: k_quant_rows_rope<256><<<resident_grid(k_quant_rows_rope<256>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int hifa4_rope_table(double theta, int pos0, int N, int d, float* cos_out, float* sin_out) {
+  if (!cos_out || !sin_out || !(theta > 1.0) || N <= 0 || pos0 < 0 || !d_ok(d)) return HIFA4_ERR_INVALID_ARG;
+  const int half = d / 2;
+  for (int i = 0; i < half; ++i) {
+    const double inv = std::pow(theta, -2.0 * i / d);
+    for (int n = 0; n < N; ++n) {
+      const double ang = (double)(pos0 + n) * inv;
+      cos_out[(long long)n * half + i] = (float)std::cos(ang);
+      sin_out[(long long)n * half + i] = (float)std::sin(ang);
+    }
+  }
+  return HIFA4_OK;
 }
 
 int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, int N, int d,
@@ -302,8 +397,10 @@ int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   const int rows = d == 256 ? 64 : 128;
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
+                   nullptr, nullptr, 0, 0,
                    static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
+                   nullptr, nullptr, 0, 0,
                    static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
   QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
                  static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 64)};
@@ -319,27 +416,87 @@ int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_
 int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
                              int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
                              void* l_out, int* status, cudaStream_t stream) {
-  if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
+  return attn_dispatch<false>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream, 0,
+                              nullptr);
+}
+
+int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq,
+                            int Hkv, int N, int d, int causal, int kv_tile, int normaliser, float* trace, void* o,
+                            void* m_out, void* l_out, int* status, cudaStream_t stream) {
+  if (normaliser != 0 && normaliser != 1) return HIFA4_ERR_INVALID_ARG;
+  if (trace && !aligned16(trace)) return HIFA4_ERR_INVALID_ARG;
+  return attn_dispatch<true>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream,
+                             normaliser, trace);
+}
+
+int hifa4_quantize_q_decode(const void* q, const int64_t q_strides[3], int B, int Hq, int Hkv, int nq, int d,
+                            const float* s, const hifa4_qtensor* q_out, int* status, cudaStream_t stream) {
+  if (!strides_ok(q, q_strides) || !status || (s && !aligned16(s))) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || (Hq / Hkv) * nq > 128 || !d_ok(d))
+    return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q_out, B, Hkv, 128, d, 0)) return HIFA4_ERR_INVALID_ARG;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  const int rows = d == 256 ? 64 : 128;
+  QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hkv, Hkv, 128, s,
+                   nullptr, nullptr, Hq / Hkv, nq, static_cast<uint8_t*>(q_out->codes),
+                   static_cast<uint8_t*>(q_out->scales), B * Hkv * (128 / rows)};
+  switch (d) {
+    case 64: k_quant_q_decode<64><<<resident_grid(k_quant_q_decode<64>, 256, qa.units), 256, 0, stream>>>(qa, status); break;
+    case 128: k_quant_q_decode<128><<<resident_grid(k_quant_q_decode<128>, 256, qa.units), 256, 0, stream>>>(qa, status); break;
+    default: k_quant_q_decode<256><<<resident_grid(k_quant_q_decode<256>, 256, qa.units), 256, 0, stream>>>(qa, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+size_t hifa4_decode_workspace_bytes(int B, int Hkv, int nsplit, int d) {
+  if (B <= 0 || Hkv <= 0 || nsplit <= 0 || nsplit > 64 || !d_ok(d)) return 0;
+  return (size_t)B * Hkv * nsplit * 128 * (d + 2) * sizeof(float);
+}
+
+int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
+                      int nq, int Nk, int d, int kv_tile, int nsplit, void* workspace, size_t workspace_bytes, void* o,
+                      void* m_out, void* l_out, int* status, cudaStream_t stream) {
+  if (!o || !status || !workspace || !aligned16(o) || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || (Hq / Hkv) * nq > 128 || Nk <= 0 || Nk % 128 ||
+      Nk > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (kv_tile == 0) kv_tile = (d == 256) ? 64 : (d == 128 ? 256 : 128);
   if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (d == 64 && kv_tile == 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (N % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (!qt_ok(q, B, Hq, N, d, 0) || !qt_ok(k, B, Hkv, N, d, 0) || !qt_ok(vt, B, Hkv, N, d, 1))
+  if ((d == 256 && kv_tile != 64) || (d == 64 && kv_tile == 256) || Nk % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (!qt_ok(q, B, Hkv, 128, d, 0) || !qt_ok(k, B, Hkv, Nk, d, 0) || !qt_ok(vt, B, Hkv, Nk, d, 1))
     return HIFA4_ERR_INVALID_ARG;
-  if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
-  if (d == 64) {
-    return kv_tile == 64 ? launch_attn<64, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
-                         : launch_attn<64, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
-  } else if (d == 128) {
-    if (kv_tile == 256) return launch_attn<128, 256>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
-    return kv_tile == 64 ? launch_attn<128, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream)
-                         : launch_attn<128, 128>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
+  const int ntile = Nk / kv_tile;
+  if (nsplit <= 0) {   // enough (batch, kv head, split) units for two waves over the SMs
+    const int want = (2 * num_sms() + B * Hkv - 1) / (B * Hkv);
+    nsplit = want < 64 ? want : 64;
   }
-  return launch_attn<256, 64>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream);
+  if (nsplit > 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (nsplit > ntile) nsplit = ntile;
+  const int tps = (ntile + nsplit - 1) / nsplit;
+  nsplit = (ntile + tps - 1) / tps;   // no empty splits (an empty split has weight 0 in the merge)
+  if (workspace_bytes < hifa4_decode_workspace_bytes(B, Hkv, nsplit, d)) return HIFA4_ERR_INVALID_ARG;
+  float* part_o = static_cast<float*>(workspace);
+  float* part_m = part_o + (size_t)B * Hkv * nsplit * 128 * d;
+  float* part_l = part_m + (size_t)B * Hkv * nsplit * 128;
+  DecodeSpec spec{nq, Hq / Hkv, Nk, nsplit, tps, part_o, part_m, part_l};
+  int rc;
+#define HIFA4_DEC(DD, BB) \
+  launch_attn<DD, BB, false, true>(q, k, vt, B, Hq, Hkv, 128, 0, o, nullptr, nullptr, status, stream, 0, nullptr, &spec)
+  if (d == 64) rc = kv_tile == 64 ? HIFA4_DEC(64, 64) : HIFA4_DEC(64, 128);
+  else if (d == 128) rc = kv_tile == 256 ? HIFA4_DEC(128, 256) : (kv_tile == 64 ? HIFA4_DEC(128, 64) : HIFA4_DEC(128, 128));
+  else rc = HIFA4_DEC(256, 64);
+#undef HIFA4_DEC
+  if (rc != HIFA4_OK) return rc;
+  DecodeMergeArgs ma{part_o, part_m, part_l, static_cast<__nv_bfloat16*>(o), static_cast<__half*>(m_out),
+                     static_cast<__half*>(l_out), Hkv, Hq / Hkv, nq, nsplit};
+  const unsigned grid = (unsigned)(B * Hkv * (Hq / Hkv) * nq);
+  switch (d) {
+    case 64: k_decode_merge<64><<<grid, 64, 0, stream>>>(ma); break;
+    case 128: k_decode_merge<128><<<grid, 128, 0, stream>>>(ma); break;
+    default: k_decode_merge<256><<<grid, 256, 0, stream>>>(ma); break;
+  }
+  return cuda_status(cudaGetLastError());
 }
 
 size_t hifa4_attn_workspace_bytes(int B, int Hkv, int N, int d) {

@@ -16,6 +16,9 @@ struct QuantRowsArgs {
   long long sb, sh, sn;
   int H, Hkv, N;
   const float* scale;         // [Hkv, D] or nullptr
+  const float* rope_cos;      // [N, D/2] fp32 angle tables of the fused RoPE path, or nullptr
+  const float* rope_sin;
+  int pack_G, pack_nq;        // decode packing (0 = off): see quant_rows_unit
   uint8_t* codes;             // [B, H, N, D/2]
   uint8_t* sf;                // [B, H, N/128, D/64, 512]
   int units;                  // B * H * N / ROWS (ROWS rows of one head per unit)
@@ -42,7 +45,16 @@ struct RowsUnit {
 // the scale from the amax and its reciprocal from a shared table, 8 code bytes stored at
 // once.  The four blocks of a 64-wide chunk sit in lanes 4q..4q+3, which assemble the
 // chunk's scale word with two shuffles.
-template <int D>
+//
+// ROPE: the rows are pre-RoPE; each thread also loads the partner block of its rotate-half
+// pair (channel c pairs with c +- D/2) and the angle table row of its token, and rotates
+// in fp32 with each product and sum rounded once:
+//   x'_c = RN(RN(x_c cos) - RN(x_{c+D/2} sin)),  x'_{c+D/2} = RN(RN(x_{c+D/2} cos) + RN(x_c sin)),
+// before Smooth-QK (which the HiFA4 abstract applies after RoPE).
+//
+// PACK: the unit is the 128-row decode tile of kv head h (H = Hkv): row r < G * nq is token
+// r % nq of query head h * G + r / nq of the [B, Hq, nq, D] input, rows >= G * nq are zero.
+template <int D, bool ROPE = false, bool PACK = false>
 __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit, const float* rtab, bool& bad) {
   using U = RowsUnit<D>;
   const int lane = threadIdx.x & 31;
@@ -52,12 +64,33 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
   const int bh = unit / per_head, n0 = (unit % per_head) * U::ROWS;
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
   const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + blk * 16;
+  constexpr int HB = U::BPR / 2;                      // blocks per half row
+  const bool first_half = blk < HB;
   uint4 raw[U::PASSES][2];
+  uint4 praw[ROPE ? U::PASSES : 1][2];
 #pragma unroll
   for (int k = 0; k < U::PASSES; ++k) {
-    const uint4* src = reinterpret_cast<const uint4*>(base + (long long)(n0 + rsub + k * U::RPP) * a.sn);
+    const int rr = n0 + rsub + k * U::RPP;
+    if constexpr (PACK) {
+      if (rr < a.pack_G * a.pack_nq) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + b * a.sb + (long long)(h * a.pack_G + rr / a.pack_nq) * a.sh +
+                                                          (long long)(rr % a.pack_nq) * a.sn + blk * 16);
+        raw[k][0] = src[0];
+        raw[k][1] = src[1];
+      } else {
+        raw[k][0] = make_uint4(0, 0, 0, 0);
+        raw[k][1] = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(base + (long long)rr * a.sn);
     raw[k][0] = src[0];
     raw[k][1] = src[1];
+    if constexpr (ROPE) {
+      const uint4* ps = src + (first_half ? 2 * HB : -2 * HB);   // the partner block, D/2 channels away
+      praw[k][0] = ps[0];
+      praw[k][1] = ps[1];
+    }
   }
   float2 s2[8];
   if (a.scale) {
@@ -76,6 +109,30 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     float2 v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
+    if constexpr (ROPE) {
+      const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&praw[k][0]);
+      const int tc = (blk % HB) * 16;                   // table column of the block's first channel
+      const float4* cp = reinterpret_cast<const float4*>(a.rope_cos + (long long)row * (D / 2) + tc);
+      const float4* sp = reinterpret_cast<const float4*>(a.rope_sin + (long long)row * (D / 2) + tc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 c4 = __ldg(cp + q), s4 = __ldg(sp + q);
+        const float2 cs[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
+        const float2 sn[2] = {make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)};
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          // scalar intrinsics: each product is rounded before the sum (never contracted into
+          // an fma, which would turn an exact cancellation into a signed rounding residue)
+          const int e = 2 * q + t;
+          const float2 y = __bfloat1622float2(q2[e]);
+          const float2 cc = cs[t], ss = sn[t];
+          const float ax = __fmul_rn(v[e].x, cc.x), ay = __fmul_rn(v[e].y, cc.y);
+          const float bx = __fmul_rn(y.x, ss.x), by = __fmul_rn(y.y, ss.y);
+          v[e] = first_half ? make_float2(__fsub_rn(ax, bx), __fsub_rn(ay, by))
+                            : make_float2(__fadd_rn(ax, bx), __fadd_rn(ay, by));
+        }
+      }
+    }
     if (a.scale) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], s2[e]);
@@ -112,6 +169,32 @@ __global__ void __launch_bounds__(256) k_quant_rows(QuantRowsArgs qa, QuantRowsA
   for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
     if (u < qa.units) quant_rows_unit<D>(qa, u, rtab, bad);
     else quant_rows_unit<D>(ka, u - qa.units, rtab, bad);
+  }
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+}
+
+// Decode Q packing + Smooth-QK + quantise: one 128-row unit per (batch, kv head).
+template <int D>
+__global__ void __launch_bounds__(256) k_quant_q_decode(QuantRowsArgs qa, int* status) {
+  __shared__ float rtab[256];
+  fill_recip_table(rtab, threadIdx.x, 256);
+  __syncthreads();
+  bool bad = false;
+  for (int u = blockIdx.x; u < qa.units; u += gridDim.x) quant_rows_unit<D, false, true>(qa, u, rtab, bad);
+  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+}
+
+// Fused RoPE + Smooth-QK + quantise of Q and K (pre-RoPE inputs), grid-stride over Q units
+// then K units.
+template <int D>
+__global__ void __launch_bounds__(256, 2) k_quant_rows_rope(QuantRowsArgs qa, QuantRowsArgs ka, int* status) {
+  __shared__ float rtab[256];
+  fill_recip_table(rtab, threadIdx.x, 256);
+  __syncthreads();
+  bool bad = false;
+  for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
+    if (u < qa.units) quant_rows_unit<D, true>(qa, u, rtab, bad);
+    else quant_rows_unit<D, true>(ka, u - qa.units, rtab, bad);
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }

@@ -49,8 +49,14 @@ def lib():
             "hifa4_calibrate_smooth": ([P, P, P, P, i, i, i, i, i, f, P, P, P, P], i),
             "hifa4_quantize_qk": ([P, P, P, P, i, i, i, i, i, P, P, QP, QP, P, P], i),
             "hifa4_quantize_v": ([P, P, i, i, i, i, QP, P, P], i),
+            "hifa4_quantize_qk_rope": ([P, P, P, P, i, i, i, i, i, P, P, P, P, QP, QP, P, P], i),
+            "hifa4_rope_table": ([ctypes.c_double, i, i, i, P, P], i),
             "hifa4_quantize_qkv": ([P, P, P, P, P, P, i, i, i, i, i, P, P, QP, QP, QP, P, P], i),
             "hifa4_attn_fwd_quantized": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
+            "hifa4_attn_fwd_ablation": ([QP, QP, QP, i, i, i, i, i, i, i, i, P, P, P, P, P, P], i),
+            "hifa4_quantize_q_decode": ([P, P, i, i, i, i, i, P, QP, P, P], i),
+            "hifa4_decode_workspace_bytes": ([i, i, i, i], sz),
+            "hifa4_attn_decode": ([QP, QP, QP, i, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
             "hifa4_attn_workspace_bytes": ([i, i, i, i], sz),
             "hifa4_attn_fwd": ([QP, QP, P, P, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
             "hifa4_read_status": ([P, i, P], i),
@@ -155,6 +161,30 @@ def hifa4_quantize_qk(q, k, s=None, sinv=None, status=None, out=None):
     return out
 
 
+def hifa4_rope_table(theta: float, N: int, d: int, pos0: int = 0):
+    """Host fp32 angle tables (cos, sin) [N, d/2] of positions pos0..pos0+N-1 (numpy)."""
+    import numpy as np
+    cos = np.empty((N, d // 2), np.float32)
+    sin = np.empty((N, d // 2), np.float32)
+    _check(lib().hifa4_rope_table(float(theta), int(pos0), N, d, cos.ctypes.data_as(ctypes.c_void_p),
+                                  sin.ctypes.data_as(ctypes.c_void_p)), "hifa4_rope_table")
+    return cos, sin
+
+
+def hifa4_quantize_qk_rope(q, k, rope_cos, rope_sin, s=None, sinv=None, status=None, out=None):
+    """Fused RoPE + Smooth-QK + 4-bit quantisation of PRE-RoPE bf16 Q [B,Hq,N,d] and K
+    [B,Hkv,N,d]; rope_cos, rope_sin: device fp32 [N, d/2] -> (QTensor, QTensor)."""
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device))
+    st = status if status is not None else new_status(q.device)
+    _check(lib().hifa4_quantize_qk_rope(_ptr(q), _ptr(k), _strides(q), _strides(k), B, Hq, Hkv, N, d, _ptr(rope_cos),
+                                        _ptr(rope_sin), _ptr(s), _ptr(sinv), out[0].c(), out[1].c(), _ptr(st),
+                                        _stream()), "hifa4_quantize_qk_rope")
+    return out
+
+
 def hifa4_quantize_qkv(q, k, v, s=None, sinv=None, status=None, out=None):
     """Smooth-QK + 4-bit Q, K and V^T in one launch -> (QTensor, QTensor, QTensor)."""
     B, Hq, N, d = q.shape
@@ -195,6 +225,55 @@ def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=
     _check(lib().hifa4_attn_fwd_quantized(qq.c(), kq.c(), vt.c(), qq.B, qq.H, kq.H, qq.N, qq.d, int(causal),
                                           int(kv_tile), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
            "hifa4_attn_fwd_quantized")
+    return o, m, l
+
+
+def hifa4_attn_fwd_ablation(q: QTensor, k: QTensor, vt: QTensor, causal: bool, kv_tile: int = 0, normaliser: int = 0,
+                            trace=None, status=None, o=None, m=None, l=None):
+    """Ablation form of the attention (see include/hifa4.h): normaliser 0 = HiFA4 (sum
+    P_hat), 1 = the inconsistent formulation (sum of unquantised P).  trace: optional fp32
+    [B, Hq, N, N/kv_tile, 2] receiving (sum P_hat, sum P) per (row, tile)."""
+    import torch
+    dev = q.codes.device
+    o = o if o is not None else torch.empty(q.B, q.H, q.N, q.d, dtype=torch.bfloat16, device=dev)
+    m = m if m is not None else torch.empty(q.B, q.H, q.N, dtype=torch.float16, device=dev)
+    l = l if l is not None else torch.empty(q.B, q.H, q.N, dtype=torch.float16, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(lib().hifa4_attn_fwd_ablation(q.c(), k.c(), vt.c(), q.B, q.H, k.H, q.N, q.d, int(causal), int(kv_tile),
+                                         int(normaliser), _ptr(trace), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
+           "hifa4_attn_fwd_ablation")
+    return o, m, l
+
+
+def hifa4_quantize_q_decode(q, Hkv: int, s=None, status=None, out=None):
+    """Smooth-QK + 4-bit quantisation of a decode query bf16 [B, Hq, nq, d] into the packed
+    [B, Hkv, 128, d] QTensor (row hi * nq + t = token t of query head g * G + hi)."""
+    B, Hq, nq, d = q.shape
+    out = out if out is not None else QTensor(B, Hkv, 128, d, 0, q.device)
+    st = status if status is not None else new_status(q.device)
+    _check(lib().hifa4_quantize_q_decode(_ptr(q), _strides(q), B, Hq, Hkv, nq, d, _ptr(s), out.c(), _ptr(st),
+                                         _stream()), "hifa4_quantize_q_decode")
+    return out
+
+
+def hifa4_attn_decode(q: QTensor, k: QTensor, vt: QTensor, Hq: int, nq: int, kv_tile: int = 0, nsplit: int = 0,
+                      status=None, workspace=None, o=None, m=None, l=None):
+    """Decode / split-KV attention of the packed query q against K, V^T of Nk = k.N keys ->
+    (o bf16 [B, Hq, nq, d], m, l fp16 [B, Hq, nq])."""
+    import torch
+    dev = q.codes.device
+    B, Hkv, Nk, d = k.B, k.H, k.N, k.d
+    ns = nsplit if nsplit > 0 else 64
+    need = lib().hifa4_decode_workspace_bytes(B, Hkv, ns, d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    o = o if o is not None else torch.empty(B, Hq, nq, d, dtype=torch.bfloat16, device=dev)
+    m = m if m is not None else torch.empty(B, Hq, nq, dtype=torch.float16, device=dev)
+    l = l if l is not None else torch.empty(B, Hq, nq, dtype=torch.float16, device=dev)
+    st = status if status is not None else new_status(dev)
+    _check(lib().hifa4_attn_decode(q.c(), k.c(), vt.c(), B, Hq, Hkv, nq, Nk, d, int(kv_tile), int(nsplit),
+                                   _ptr(workspace), workspace.numel(), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
+           "hifa4_attn_decode")
     return o, m, l
 
 

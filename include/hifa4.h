@@ -131,6 +131,34 @@ HIFA4_API int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B,
                      const hifa4_qtensor* vt_out, int* status, cudaStream_t stream);
 
 /*
+ * Fused RoPE + Smooth-QK + 4-bit quantisation of Q and K (the step before the attention:
+ * the HiFA4 abstract applies the per-channel rescaling after RoPE, so the rotation, the
+ * rescaling and the quantisation run in one pass over the pre-RoPE tensors).
+ * q, k: bf16 [B, Hq, N, d] / [B, Hkv, N, d] BEFORE RoPE, strides as for hifa4_quantize_qk.
+ * rope_cos, rope_sin: device fp32 [N, d/2], 16-byte aligned; row n holds the angles of
+ * token n (its position), column i those of channel pair (i, i + d/2).  Rotate-half RoPE
+ * in fp32, each product and the sum rounded once:
+ *   x'_i = RN(RN(x_i cos) - RN(x_{i+d/2} sin)),  x'_{i+d/2} = RN(RN(x_{i+d/2} cos) + RN(x_i sin)),
+ * then q' = RN(x' * s[g,c]) (k' with sinv) and the 16-element block quantiser of
+ * hifa4_quantize_qk; the rotated values are not rounded to bf16.  Same outputs and errors
+ * as hifa4_quantize_qk (HIFA4_ERR_INVALID_ARG also for a missing or misaligned table).
+ */
+HIFA4_API int hifa4_quantize_qk_rope(const void* q, const void* k, const int64_t q_strides[3],
+                                     const int64_t k_strides[3], int B, int Hq, int Hkv, int N, int d,
+                                     const float* rope_cos, const float* rope_sin, const float* s, const float* sinv,
+                                     const hifa4_qtensor* q_out, const hifa4_qtensor* k_out, int* status,
+                                     cudaStream_t stream);
+
+/*
+ * Host helper: the angle tables of hifa4_quantize_qk_rope for positions pos0 .. pos0+N-1,
+ * inv_freq_i = theta^(-2i/d), angle = position * inv_freq_i, cos and sin computed in double
+ * and rounded once to fp32.  cos_out, sin_out: HOST fp32 [N, d/2] (caller-owned; copy them
+ * to the device).  Returns HIFA4_ERR_INVALID_ARG for null outputs, theta <= 1, N <= 0,
+ * pos0 < 0 or an unsupported d.
+ */
+HIFA4_API int hifa4_rope_table(double theta, int pos0, int N, int d, float* cos_out, float* sin_out);
+
+/*
  * hifa4_quantize_qk and hifa4_quantize_v in one launch (same arguments and outputs; the
  * three quantisations are independent, so V's latency hides behind Q and K).
  */
@@ -148,9 +176,10 @@ HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, co
  *   m_new  = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e) / sqrt(d))
  *   P      = E(RN(fma(S, c, -m_new)))            (E: the library's deterministic exp2)
  *   P_hat  = 4-bit blocks of 16 keys, each block's scale sigma from E(fma(blockmax S, c,
- *            -m_new)); a score's code is the E2M1 rounding of y = p(frac(128u)) *
- *            2^(floor(128u) - 125), u = sat(S c/128 + (RN(-log2 sigma) - m_new + 125)/128),
- *            i.e. of P / sigma evaluated in the log domain
+ *            -m_new)); a score's code is the E2M1 rounding of y = 2^floor(z) (1 + frac z),
+ *            z = 128u - 125 - 73/1024 on a 2^-10 grid, u = sat(S c/128 + (RN(-log2 sigma)
+ *            - m_new + 125)/128): P / sigma evaluated in the log domain with a linear
+ *            mantissa (rounding boundaries within 1% of the exact exponential's)
  *   alpha  = E(m - m_new)  (0 on the first tile)
  *   O      = alpha * O + P_hat V_hat_j           (4-bit MMA)
  *   r      = P_hat * 1                           (4-bit MMA against ones: P-Reordering)
@@ -163,6 +192,58 @@ HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, co
 HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
                              int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
                              void* l_out, int* status, cudaStream_t stream);
+
+/*
+ * Ablation form of hifa4_attn_fwd_quantized (same arguments, outputs and errors, plus
+ * two): the kernel also sums the unquantised P = E(RN(fma(S, c, -m_new))) of every row and
+ * kv tile in fp32 (each 64-column (Bc = 64: 32-column) chunk of the row in order, then the
+ * chunks in order).
+ *   normaliser 0: l from r = P_hat * 1 as in HiFA4 (O, m, l identical to
+ *                 hifa4_attn_fwd_quantized);
+ *   normaliser 1: l from r = sum P, the "inconsistent formulation" of the HiFA4 abstract
+ *                 (PV still uses P_hat), i.e. each tile's contribution to O is scaled by
+ *                 sum P_hat / sum P.  With Q and K quantised without Smooth-QK (s = NULL)
+ *                 this is the abstract's "direct HIF4 quantization" baseline.
+ * trace: device fp32 [B, Hq, N, N / kv_tile, 2] (16-byte aligned) or NULL; entry (row,
+ *   tile, 0) = sum P_hat (exact), (row, tile, 1) = sum P of that tile, for every tile the
+ *   row's 128-row query tile visits (causal: later tiles are not written; a visited tile
+ *   with no visible key for the row holds 0, 0).  The per-tile mass error of the abstract
+ *   is eps = sum P_hat / sum P - 1.
+ * HIFA4_ERR_INVALID_ARG for normaliser outside {0, 1} or a misaligned trace.
+ */
+HIFA4_API int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt,
+                                      int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, int normaliser,
+                                      float* trace, void* o, void* m_out, void* l_out, int* status,
+                                      cudaStream_t stream);
+
+/*
+ * Decode / split-KV attention: a short query (nq tokens per sequence, the last nq positions)
+ * against Nk keys of 4-bit K and V^T (a KV cache quantised with hifa4_quantize_qk /
+ * hifa4_quantize_v, N = Nk).  The G = Hq / Hkv query heads of a kv head and the nq tokens
+ * are packed into one 128-row tile (G * nq <= 128): row r = hi * nq + t is token t of query
+ * head g * G + hi, at position Nk - nq + t, and sees the keys <= that position.
+ *
+ * hifa4_quantize_q_decode: Smooth-QK (s, NULL = off) and 4-bit quantisation of bf16
+ *   q [B, Hq, nq, d] (strides as for hifa4_quantize_qk) into the packed q_out, a
+ *   transposed == 0 tensor of sizes [B, Hkv, 128, d] (rows >= G * nq are zero).
+ * hifa4_attn_decode: the Nk / kv_tile kv tiles are cut into nsplit runs of
+ *   ceil(tiles / nsplit) tiles (nsplit <= 0: chosen from the SM count; at most 64; empty
+ *   runs are dropped, which the merge would weight 0).  Every (batch, kv head, run) runs the
+ *   HiFA4 tile loop of hifa4_attn_fwd_quantized from the initial state and leaves (m_s, l_s,
+ *   unnormalised fp32 O_s) in `workspace` (hifa4_decode_workspace_bytes(B, Hkv, nsplit, d)
+ *   bytes, 16-byte aligned); a second launch merges in fp32, runs in order:
+ *     m = max m_s,  w_s = E(m_s - m) (0 for m_s = -inf),  L = fma(w_s, l_s, L),
+ *     O = fma(w_s, O_s, O),  out = bf16_RN(O * RN(1/L)).
+ *   o: bf16 [B, Hq, nq, d] dense; m_out, l_out: fp16 [B, Hq, nq] (m, RN(L)) or NULL.
+ *   Nk a multiple of 128 and of kv_tile; kv_tile as for hifa4_attn_fwd_quantized.
+ */
+HIFA4_API int hifa4_quantize_q_decode(const void* q, const int64_t q_strides[3], int B, int Hq, int Hkv, int nq, int d,
+                                      const float* s, const hifa4_qtensor* q_out, int* status, cudaStream_t stream);
+HIFA4_API size_t hifa4_decode_workspace_bytes(int B, int Hkv, int nsplit, int d);
+HIFA4_API int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq,
+                                int Hkv, int nq, int Nk, int d, int kv_tile, int nsplit, void* workspace,
+                                size_t workspace_bytes, void* o, void* m_out, void* l_out, int* status,
+                                cudaStream_t stream);
 
 /*
  * The full attention forward on quantised Q, K and bf16 V: quantises V^T into

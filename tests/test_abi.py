@@ -75,3 +75,17 @@ def test_layout_permutations_roundtrip():
         pv = rng.integers(0, 256, (B, H, dd, N // 16), dtype=np.uint8)
         av = _layout.vt_scales_from_plain(pv, B, H, N, dd)
         assert np.array_equal(_layout.vt_scales_to_plain(av, B, H, N, dd), pv)
+
+
+def test_rope_table_matches_float64_angles():
+    # host helper, no GPU: cos/sin of position * theta^(-2i/d) in double, rounded once
+    from bit_flashattention_b200 import hifa4
+    N, d, theta, pos0 = 300, 128, 5e5, 9
+    cos, sin = hifa4.hifa4_rope_table(theta, N, d, pos0=pos0)
+    inv = theta ** (-np.arange(0, d // 2, dtype=np.float64) * 2.0 / d)
+    ang = (pos0 + np.arange(N, dtype=np.float64))[:, None] * inv[None, :]
+    for got, ref in ((cos, np.cos(ang)), (sin, np.sin(ang))):
+        ulp = np.spacing(np.abs(ref.astype(np.float32)))
+        assert np.all(np.abs(got.astype(np.float64) - ref) <= 0.5 * ulp + 1e-12)
+    with pytest.raises(hifa4.Hifa4Error):
+        hifa4.hifa4_rope_table(1.0, N, d)
