@@ -134,6 +134,70 @@ def make_inputs(w, device):
     return sets, host, s, sinv
 
 
+# Decode / split-KV measurement: a 4-bit KV cache of DECODE_NK keys for DECODE_B sequences
+# with the Qwen3-8B head layout; one step = quantise the packed query of nq new tokens per
+# sequence (hifa4_quantize_q_decode) + hifa4_attn_decode (split attention + merge).
+DECODE_B, DECODE_NK = 16, 32768
+
+
+def measure_decode(hifa4, torch, device, steps, dist):
+    B, Hq, Hkv, d, Nk = DECODE_B, 32, 8, 128, DECODE_NK
+    gen_ = torch.Generator(device=device)
+    gen_.manual_seed(20261202)
+    st = hifa4.new_status(device)
+    kq = hifa4.QTensor(B, Hkv, Nk, d, 0, device)
+    vq = hifa4.QTensor(B, Hkv, Nk, d, 1, device)
+    kc_b, ks_b = kq.codes.numel() // B, kq.scales.numel() // B
+    vc_b, vs_b = vq.codes.numel() // B, vq.scales.numel() // B
+    qdummy = hifa4.QTensor(4, Hkv, Nk, d, 0, device)
+    for b0 in range(0, B, 4):   # quantise the cache in slices of 4 sequences (bounded bf16 scratch)
+        kb = torch.randn(4, Hkv, Nk, d, generator=gen_, device=device, dtype=torch.float32).to(torch.bfloat16)
+        vb = torch.randn(4, Hkv, Nk, d, generator=gen_, device=device, dtype=torch.float32).to(torch.bfloat16)
+        ks = hifa4.QTensor(4, Hkv, Nk, d, 0, codes=kq.codes[b0 * kc_b:(b0 + 4) * kc_b],
+                           scales=kq.scales[b0 * ks_b:(b0 + 4) * ks_b])
+        vs = hifa4.QTensor(4, Hkv, Nk, d, 1, codes=vq.codes[b0 * vc_b:(b0 + 4) * vc_b],
+                           scales=vq.scales[b0 * vs_b:(b0 + 4) * vs_b])
+        hifa4.hifa4_quantize_qk(kb, kb, status=st, out=(qdummy, ks))
+        hifa4.hifa4_quantize_v(vb, status=st, out=vs)
+        del kb, vb
+    del qdummy
+    kv_bytes = 2 * B * Hkv * Nk * d * (0.5 + 1 / 16)
+    out = {"B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "Nk": Nk, "kv_tile": 256, "nsplit": "auto",
+           "kv_cache_bytes": kv_bytes}
+    ws = None
+    for nq in (1, 32):
+        q = torch.randn(B, Hq, nq, d, generator=gen_, device=device, dtype=torch.float32).to(torch.bfloat16)
+        qp = hifa4.QTensor(B, Hkv, 128, d, 0, device)
+        o = torch.empty(B, Hq, nq, d, dtype=torch.bfloat16, device=device)
+        if ws is None:
+            ws = torch.empty(hifa4.lib().hifa4_decode_workspace_bytes(B, Hkv, 64, d), dtype=torch.uint8, device=device)
+
+        def dstep():
+            hifa4.hifa4_quantize_q_decode(q, Hkv, status=st, out=qp)
+            hifa4.hifa4_attn_decode(qp, kq, vq, Hq, nq, kv_tile=256, nsplit=0, status=st, workspace=ws, o=o)
+
+        for _ in range(3):
+            dstep()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(steps):
+            dstep()
+        e1.record()
+        torch.cuda.synchronize()
+        if hifa4.hifa4_read_status(st) != hifa4.OK:
+            raise RuntimeError("decode reported an error")
+        us = e0.elapsed_time(e1) / steps * 1e3
+        us = reduce_max(us, dist, device)
+        out[f"nq{nq}"] = {"us_per_step": round(us, 2), "tokens_per_s": round(B * nq / (us * 1e-6), 1),
+                          "kv_gbs": round(kv_bytes / (us * 1e-6) / 1e9, 1),
+                          "attn_tflops": round(4.0 * B * Hq * nq * Nk * d / (us * 1e-6) / 1e12, 2)}
+    out["note"] = ("step = packed-query quantiser + split attention + merge; kv_gbs = 4-bit K and V^T "
+                   "(codes + scales) bytes / step time; the 0.6 GB cache exceeds L2")
+    return out
+
+
 def run_gpu(args):
     import torch
     from bit_flashattention_b200 import configs, hifa4
@@ -257,6 +321,7 @@ def run_gpu(args):
     k_attn = reduce_max(k_attn, dist, device)
     k_quant = reduce_max(k_quant, dist, device)
     k_rope = reduce_max(k_rope, dist, device)
+    decode = measure_decode(hifa4, torch, device, max(20, min(args.steps, 200)), dist)
     agg = aggregate([elapsed] * world, flops, args.steps)
     e2e = aggregate([e2e_ms] * world, flops, e2e_steps)
     h2d = sum(x.numel() * x.element_size() for x in host)
@@ -293,6 +358,7 @@ def run_gpu(args):
         "attn_kernel_tflops": round(achieved, 2),
         "quantize_qkv_gbs": round(quant_bytes / (k_quant * 1e-3) / 1e9, 1),
         "quantize_qkv_frac_hbm": round(quant_bytes / (k_quant * 1e-3) / 1e9 / hbm, 3),
+        "decode": decode,
         "quantize_qk_rope": {"us": round(k_rope * 1e3, 2), "launches": n_rope,
                              "gbs": round(rope_bytes / (k_rope * 1e-3) / 1e9, 1),
                              "frac_hbm": round(rope_bytes / (k_rope * 1e-3) / 1e9 / hbm, 3),
