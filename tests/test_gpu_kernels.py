@@ -173,3 +173,37 @@ def test_pv_mma_probe(d, bc):
     ref = P @ V.T
     assert np.max(np.abs(O - ref)) <= 1e-5 * max(1.0, np.abs(ref).max())
     assert np.array_equal(R, P.sum(1))          # the normaliser column is exact
+
+
+def test_quantize_qkv_strided_and_full_size():
+    # the one-launch quantiser (TMA-fed): permuted [B, N, H, d] views of Q, K, V, and the
+    # full qwen3-8b-4k tensors of the benchmark, bit-exact against the oracle
+    w = configs.scaled(configs.get("qwen3-8b-4k"), B=2, Hq=4, Hkv=2, N=256)
+    q, k, v = gen.inputs(w)
+    views = [gc.bf16_dev(np.ascontiguousarray(x.transpose(0, 2, 1, 3))).permute(0, 2, 1, 3) for x in (q, k, v)]
+    assert not views[0].is_contiguous()
+    s, sinv = gc.smooth_scales(w)
+    st = hifa4.new_status("cuda")
+    qq, kq, vq = hifa4.hifa4_quantize_qkv(*views, gc.to_dev(s), gc.to_dev(sinv), status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    res = gc.oracle_from_gpu_layout_check(w, qq, kq, vq, oracle.quantize_all(q, k, v, s, sinv))
+    assert all(res.values()), res
+
+    w = configs.get("qwen3-8b-4k")
+    q, k, v = gen.inputs(w)
+    s, sinv = gc.smooth_scales(w)
+    qq, kq, vq = hifa4.hifa4_quantize_qkv(gc.bf16_dev(q), gc.bf16_dev(k), gc.bf16_dev(v), gc.to_dev(s),
+                                          gc.to_dev(sinv), status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    res = gc.oracle_from_gpu_layout_check(w, qq, kq, vq, oracle.quantize_all(q, k, v, s, sinv))
+    assert all(res.values()), res
+
+
+def test_quantize_qkv_flags_nonfinite_input():
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=256)
+    q, k, v = gen.inputs(w)
+    vt = gc.bf16_dev(v)
+    vt[0, 0, 77, 5] = float("inf")
+    st = hifa4.new_status("cuda")
+    hifa4.hifa4_quantize_qkv(gc.bf16_dev(q), gc.bf16_dev(k), vt, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.ERR_NONFINITE
