@@ -29,6 +29,12 @@
  *     l = fp16_RN(fma(alpha, l, r)), r = exact sum of the tile's P_hat,
  *     O = alpha*O (fp32) + (exact tile P_hat V_hat rounded to fp32),
  *     out = bf16_RN(RN(O / l)).
+ *   - two-level P scale (ablation variant, two_level = 1): a per-(row, tile) power of two
+ *     2^k under the block scales of P, k = max(floor(log2 p_t) - 10, -40) with p_t the
+ *     tile's largest block amax of P; sigma_b = E4M3_RN(RN(amax * RN(1/6)) * 2^-k),
+ *     P_hat = code * sigma_b * 2^k, L from the effective scale sigma_b * 2^k.  Where the
+ *     one-level scale is a normal E4M3 value both give the same P_hat; blocks too small
+ *     for one level (scale 0 or subnormal) keep their mass.
  *   - S accumulation of the 4-bit GEMM: one of the models in s_dot(), selected by the
  *     caller; the mirror uses model 3 (per 64-wide MMA step, the exact sum of the fp32
  *     accumulator and the step's block products, rounded toward zero), which is what a
@@ -150,6 +156,14 @@ static float own_exp2(float x) {
 static float neg_log2_scale(uint8_t code) {
     int e = (code >> 3) & 15, m = code & 7;
     double v = (e == 0) ? 9.0 - log2((double)m) : (double)(10 - e) - log2((double)(8 + m));
+    return (float)v;
+}
+
+/* L of the effective scale sigma * 2^k (two-level P scale): the same integer-log form with
+ * the integer part lowered by k before the one subtraction, so k = 0 is neg_log2_scale. */
+static float neg_log2_scale_k(uint8_t code, int k) {
+    int e = (code >> 3) & 15, m = code & 7;
+    double v = (e == 0) ? (double)(9 - k) - log2((double)m) : (double)(10 - e - k) - log2((double)(8 + m));
     return (float)v;
 }
 
@@ -424,6 +438,7 @@ typedef struct {
      * tile range [j0, j1) of this call, and dec_nq > 0 for packed decode rows: query row i
      * holds token i % dec_nq, at position Nk - dec_nq + (i % dec_nq), which sees keys <= it */
     int Nk, j0, j1, dec_nq;
+    int two_level;    /* 1: per-(row, tile) second-level P scale 2^k (see the header) */
 } loop_args;
 
 /* Per-row output and optional per-tile trace. */
@@ -511,14 +526,27 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
         double P[256], Ph[256];
         for (int kk = 0; kk < bc; ++kk) { P[kk] = 0.0; Ph[kk] = 0.0; }
         if (a->quant) {
+            float amaxs[16];
+            float p_t = 0.0f;                                 /* the tile's largest block amax */
             for (int blk = 0; blk < bc / 16; ++blk) {
                 float bmax = -INFINITY;
                 for (int e = 0; e < 16; ++e) bmax = fmaxf(bmax, Sf[blk * 16 + e]);
-                float amax = own_exp2(fmaf(bmax, c, -mref));  /* = block amax of P (E monotone) */
-                uint8_t sc = e4m3_encode_pos(amax * (1.0f / 6.0f));
-                float sigma = e4m3_value(sc);
+                amaxs[blk] = own_exp2(fmaf(bmax, c, -mref));  /* = block amax of P (E monotone) */
+                if (amaxs[blk] > p_t) p_t = amaxs[blk];
+            }
+            int k2 = 0;                                       /* second-level scale 2^k2 */
+            if (a->two_level) {
+                int ex;
+                frexpf(p_t, &ex);                             /* p_t = f 2^ex, f in [0.5, 1) */
+                k2 = (ex - 1) - 10;
+                if (p_t == 0.0f || k2 < -40) k2 = -40;
+            }
+            for (int blk = 0; blk < bc / 16; ++blk) {
+                float amax = amaxs[blk];
+                uint8_t sc = e4m3_encode_pos(ldexpf(amax * (1.0f / 6.0f), -k2));
+                float sigma = ldexpf(e4m3_value(sc), k2);
                 float B = -INFINITY;                          /* sigma == 0: every code is 0 */
-                if (sigma > 0.0f) B = ((neg_log2_scale(sc) - mref) + 125.0f) * 0.0078125f;
+                if (sigma > 0.0f) B = ((neg_log2_scale_k(sc, k2) - mref) + 125.0f) * 0.0078125f;
                 for (int e = 0; e < 16; ++e) {
                     int kk = blk * 16 + e;
                     float p = own_exp2(fmaf(Sf[kk], c, -mref));
@@ -607,16 +635,17 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
 /* Quantised attention forward over selected rows (row id = (b*Hq + h)*N + i; rows == NULL
  * means all rows in order).  state: 0 mirror (fp16 m, l), 1 fp64 state with exact 2^x.
  * l_from_p: 1 selects the inconsistent normaliser (sum of unquantised P).
+ * two_level: 1 selects the two-level P scale (see the header).
  * Outputs per selected row r: o_f64[r*d..] (may be NULL), o_bf16[r*d..] (may be NULL),
  * m_out[r], l_out[r] (fp32 holding the state value). */
 OR_EXPORT int or_attn_fwd(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
                           const uint8_t* vtc, const uint8_t* vts, int B, int Hq, int Hkv, int N, int d,
-                          int causal, int bc, int state, int l_from_p, int s_model,
+                          int causal, int bc, int state, int l_from_p, int two_level, int s_model,
                           const long long* rows, long long nrows,
                           double* o_f64, uint16_t* o_bf16, float* m_out, float* l_out) {
     if (d % 16 || d > 256 || bc % 16 || bc > 256 || N % bc || Hq % Hkv) return -1;
     loop_args a = {qc, qs, kc, ks, vtc, vts, NULL, NULL, NULL, B, Hq, Hkv, N, d, causal, bc,
-                   1, state, l_from_p, s_model};
+                   1, state, l_from_p, s_model, 0, 0, 0, 0, two_level};
     long long n = rows ? nrows : (long long)B * Hq * N;
 #pragma omp parallel for schedule(dynamic, 16)
     for (long long r = 0; r < n; ++r) {
@@ -648,11 +677,11 @@ OR_EXPORT int or_attn_loop_exact(const uint16_t* q, const uint16_t* k, const uin
 /* Per-tile trace of one row of the quantised loop (state as in or_attn_fwd). */
 OR_EXPORT int or_attn_trace(const uint8_t* qc, const uint8_t* qs, const uint8_t* kc, const uint8_t* ks,
                             const uint8_t* vtc, const uint8_t* vts, int B, int Hq, int Hkv, int N, int d,
-                            int causal, int bc, int state, int l_from_p, int s_model, long long row,
+                            int causal, int bc, int state, int l_from_p, int two_level, int s_model, long long row,
                             float* tr_m, float* tr_p, float* tr_phat, double* o_f64, float* ml) {
     if (d % 16 || d > 256 || bc % 16 || bc > 256 || N % bc || Hq % Hkv) return -1;
     loop_args a = {qc, qs, kc, ks, vtc, vts, NULL, NULL, NULL, B, Hq, Hkv, N, d, causal, bc,
-                   1, state, l_from_p, s_model};
+                   1, state, l_from_p, s_model, 0, 0, 0, 0, two_level};
     row_out o = {o_f64, NULL, 0, 0, tr_m, tr_p, tr_phat};
     row_loop(&a, row, &o);
     ml[0] = o.m;

@@ -59,11 +59,11 @@ def lib():
         L.or_attn_decode.restype = i
         L.or_quantize_rows_f32.argtypes = [P, i, i, i, i, i, P, P, P]
         L.or_qk_scores.argtypes = [P, P, P, P, i, i, i, i, P]
-        L.or_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, P, ll, P, P, P, P]
+        L.or_attn_fwd.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, P, ll, P, P, P, P]
         L.or_attn_fwd.restype = i
         L.or_attn_loop_exact.argtypes = [P, P, P, i, i, i, i, i, i, i, P, ll, P]
         L.or_attn_loop_exact.restype = i
-        L.or_attn_trace.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, ll, P, P, P, P, P]
+        L.or_attn_trace.argtypes = [P, P, P, P, P, P, i, i, i, i, i, i, i, i, i, i, i, ll, P, P, P, P, P]
         L.or_attn_trace.restype = i
         L.or_attn_bruteforce.argtypes = [P, P, P, i, i, i, i, i, i, P, ll, P]
         L.or_f16_bits.argtypes = [ctypes.c_float]
@@ -235,10 +235,11 @@ def quantize_all(q, k, v, s=None, sinv=None):
 
 
 def attn_fwd(qz: Quantized, causal, bc, rows=None, state=STATE_MIRROR, l_from_p=False,
-             s_model=S_MODEL_DEFAULT, want_f64=False):
+             s_model=S_MODEL_DEFAULT, want_f64=False, two_level=False):
     """Quantised online attention over the selected rows (all rows when rows is None).
-    Returns dict with o_bf16 [n, d] (uint16), m, l [n] (fp32 holding the state values),
-    m16 / l16 (fp16 bit patterns) and, when want_f64, o_f64 [n, d]."""
+    two_level selects the two-level P scale (a per-row, per-tile power of two under the
+    block scales of P).  Returns dict with o_bf16 [n, d] (uint16), m, l [n] (fp32 holding
+    the state values), m16 / l16 (fp16 bit patterns) and, when want_f64, o_f64 [n, d]."""
     n = qz.B * qz.Hq * qz.N if rows is None else len(rows)
     r = None if rows is None else _c(rows, np.int64)
     d = qz.d
@@ -247,8 +248,8 @@ def attn_fwd(qz: Quantized, causal, bc, rows=None, state=STATE_MIRROR, l_from_p=
     m = np.empty(n, np.float32)
     l = np.empty(n, np.float32)
     rc = lib().or_attn_fwd(_p(qz.qc), _p(qz.qs), _p(qz.kc), _p(qz.ks), _p(qz.vc), _p(qz.vs),
-                           qz.B, qz.Hq, qz.Hkv, qz.N, d, int(causal), bc, state, int(l_from_p), s_model,
-                           _p(r), n, _p(o64), _p(o16), _p(m), _p(l))
+                           qz.B, qz.Hq, qz.Hkv, qz.N, d, int(causal), bc, state, int(l_from_p), int(two_level),
+                           s_model, _p(r), n, _p(o64), _p(o16), _p(m), _p(l))
     if rc != 0:
         raise ValueError("oracle rejected the shape")
     out = {"o_bf16": o16, "m": m, "l": l,
@@ -291,7 +292,8 @@ def attn_decode(qc, qs, kc, ks, vc, vs, G, nq, bc, nsplit, s_model=S_MODEL_DEFAU
     return {"o_bf16": o, "m": m, "l": l, "part_o": po, "part_ml": pml}
 
 
-def attn_trace(qz: Quantized, causal, bc, row, state=STATE_MIRROR, l_from_p=False, s_model=S_MODEL_DEFAULT):
+def attn_trace(qz: Quantized, causal, bc, row, state=STATE_MIRROR, l_from_p=False, s_model=S_MODEL_DEFAULT,
+               two_level=False):
     """Per-tile trace of one row: m after each tile, P and dequantised P_hat per key,
     O / l in the state precision, final (m, l)."""
     i = row % qz.N
@@ -302,8 +304,8 @@ def attn_trace(qz: Quantized, causal, bc, row, state=STATE_MIRROR, l_from_p=Fals
     o = np.empty(qz.d, np.float64)
     ml = np.empty(2, np.float32)
     rc = lib().or_attn_trace(_p(qz.qc), _p(qz.qs), _p(qz.kc), _p(qz.ks), _p(qz.vc), _p(qz.vs),
-                             qz.B, qz.Hq, qz.Hkv, qz.N, qz.d, int(causal), bc, state, int(l_from_p), s_model,
-                             int(row), _p(tr_m), _p(tr_p), _p(tr_ph), _p(o), _p(ml))
+                             qz.B, qz.Hq, qz.Hkv, qz.N, qz.d, int(causal), bc, state, int(l_from_p),
+                             int(two_level), s_model, int(row), _p(tr_m), _p(tr_p), _p(tr_ph), _p(o), _p(ml))
     if rc != 0:
         raise ValueError("oracle rejected the shape")
     return {"m": tr_m, "p": tr_p.reshape(ntiles, bc), "phat": tr_ph.reshape(ntiles, bc),
