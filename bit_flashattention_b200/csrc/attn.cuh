@@ -111,7 +111,12 @@ struct AttnParams {
   float* part_m;            // [B * Hkv * nsplit * 128]
   float* part_l;
   float* trace;             // ablation kernels: [B*Hq*N][N/BC][2] per (row, tile): sum P_hat, sum P; or nullptr
+  // ablation kernels: 1 = two-level P scale, a per-(row, tile) power of two 2^k under the
+  // block scales of P, k = max(floor(log2 p_t) - 10, -40), p_t the tile's largest block
+  // amax; TMEM then holds O * 2^-k and R * 2^-k
+  int two_level;
   float lneg[128];          // L(sigma) = RN(-log2 sigma) per E4M3 scale code (-inf for 0)
+  double lg2[16];           // log2(i) in double, i = 1..15 (two-level L of sigma * 2^k)
 };
 
 // Keep the register results of tcgen05.ld from being read before tcgen05.wait::ld.
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     // split's partial).  It runs after the next unit's first tile, which touches neither O
     // nor R, so that tile's work overlaps the last PV.
     const int ntmax = p.N / BC;
-    auto epilogue = [&](int gl, long long orow, float l_e, float alpha_e, float rsum_e, int jl) -> bool {
+    auto epilogue = [&](int gl, long long orow, float l_e, float alpha_e, float rsum_e, int jl, float kpow_e) -> bool {
       if (!wait_all(o_bar, gl & 1, abort, p.status, p.wait_ns)) return false;
       tc_fence_after();
       uint32_t rr[1] = {tmem_ld1(tbase + lrow + C::T_R)};
@@ -458,6 +463,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       reg_fence(rr);
       float r_use = __uint_as_float(rr[0]);
       if constexpr (SUMP) {
+        r_use = __fmul_rn(r_use, kpow_e);   // two-level: R * 2^-k -> sum P_hat (exact)
         if (p.trace && wg == 0) {
           float* t = p.trace + (orow * ntmax + jl) * 2;
           t[0] = r_use;
@@ -487,7 +493,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         if (wg == 0) p.part_l[orow] = l_fin;
         return true;
       }
-      const float inv = (l_fin > 0.0f) ? __frcp_rn(l_fin) : 0.0f;
+      float inv = (l_fin > 0.0f) ? __frcp_rn(l_fin) : 0.0f;
+      if constexpr (SUMP) inv = __fmul_rn(inv, kpow_e);   // O in TMEM is O * 2^-k
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * D);
 #pragma unroll 1
       for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
@@ -519,6 +526,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     float pend_l = 0.0f, pend_alpha = 0.0f;
     float pend_rsum = 0.0f;                  // ablation kernels: its last tile's sum of P and index
     int pend_j = 0;
+    float pend_kpow = 1.0f;                  // two-level: 2^k of that tile
     int g = 0;   // global tile counter
     for (int i = 0, u = unit_of(0); ok && u < units; u = unit_of(++i)) {
       const UnitGeom ug = unit_geom<BC, DEC>(u, p);
@@ -535,6 +543,8 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       }
       float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
       float rsum_prev = 0.0f;                // ablation kernels: the previous tile's sum of P
+      int k_prev = 0;                        // two-level: the previous tile's k and 2^k
+      float kpow_prev = 1.0f;
       for (int jj = 0; jj < nt; ++jj, ++g) {
         const int j = ug.j0 + jj;
         const int sb = g % C::SB, pb = g & 1;
@@ -585,6 +595,20 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
             (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
         const float negm = -mnew;
         const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
+        // O is rescaled by alpha_o: alpha, times 2^(k_prev - k) with the two-level scale
+        float alpha_o = alpha, kinv = 1.0f, kpow = 1.0f;
+        int k2 = 0;
+        if constexpr (SUMP) {
+          if (p.two_level) {
+            // p_t = E(fma(rowmax S, c, -m_new)), the largest block amax of P (E monotone)
+            const float pt = exp2_own(__fmaf_rn(rmax, c, negm));
+            k2 = (int)((__float_as_uint(pt) >> 23) & 0xFFu) - 127 - 10;
+            k2 = k2 < -40 ? -40 : k2;
+            kinv = __uint_as_float((uint32_t)(127 - k2) << 23);
+            kpow = __uint_as_float((uint32_t)(127 + k2) << 23);
+            alpha_o = __fmul_rn(alpha, __uint_as_float((uint32_t)(127 + k_prev - k2) << 23));
+          }
+        }
         float rsum = 0.0f;
         if constexpr (SUMP) {
           float part = 0.0f;
@@ -612,10 +636,20 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         uint32_t sfw = 0;
 #pragma unroll
         for (int bl = 0; bl < NB; ++bl) {
-          const uint32_t sc = cvt_e4m3(__fmul_rn(pmax[bl], kSixth));
+          float sarg = __fmul_rn(pmax[bl], kSixth);
+          if constexpr (SUMP) sarg = __fmul_rn(sarg, kinv);
+          const uint32_t sc = cvt_e4m3(sarg);
           sfw |= sc << (8 * bl);
+          float Lb = rtab[sc];
+          if constexpr (SUMP) {
+            if (p.two_level && sc != 0) {
+              // L of the effective scale sigma * 2^k: the integer part lowered by k first
+              const int e4 = (int)(sc >> 3) & 15, m3 = (int)sc & 7;
+              Lb = __double2float_rn(e4 == 0 ? (double)(9 - k2) - p.lg2[m3] : (double)(10 - e4 - k2) - p.lg2[8 + m3]);
+            }
+          }
           // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-          const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
+          const float B = __fmul_rn(__fadd_rn(__fsub_rn(Lb, mnew), 125.0f), 0.0078125f);
 #pragma unroll
           for (int h8 = 0; h8 < 2; ++h8) {
             float2 y[4];
@@ -647,6 +681,7 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           reg_fence(rr);
           float r_use = __uint_as_float(rr[0]);
           if constexpr (SUMP) {
+            r_use = __fmul_rn(r_use, kpow_prev);
             if (p.trace && wg == 0) {
               float* t = p.trace + ((ug.orow + row) * ntmax + (j - 1)) * 2;
               t[0] = r_use;
@@ -655,14 +690,14 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
             if (p.l_from_p) r_use = rsum_prev;
           }
           l_run = f16_round(__fmaf_rn(alpha_prev, l_run, r_use));
-          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          if (__any_sync(0xffffffffu, alpha_o != 1.0f)) {
 #pragma unroll 1
             for (int c0 = wg * OW; c0 < wg * OW + OW; c0 += 32) {
               uint32_t o[32];
               tmem_ld32(tbase + lrow + C::T_O + c0, o);
               tmem_wait_ld();
               reg_fence(o);
-              const float2 a2 = make_float2(alpha, alpha);
+              const float2 a2 = make_float2(alpha_o, alpha_o);
 #pragma unroll
               for (int q = 0; q < 32; q += 2) {
                 const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[q]), __uint_as_float(o[q + 1])), a2);
@@ -680,8 +715,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         alpha_prev = alpha;
         m_run = mnew;
         rsum_prev = rsum;
+        k_prev = k2;
+        kpow_prev = kpow;
         if (jj == 0 && i > 0) {
-          ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j);
+          ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j, pend_kpow);
           if (!ok) break;
         }
       }
@@ -691,12 +728,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
       pend_alpha = alpha_prev;
       pend_rsum = rsum_prev;
       pend_j = ug.j0 + nt - 1;
+      pend_kpow = kpow_prev;
       if (wg == 0) {
         if constexpr (DEC) p.part_m[pend_row] = m_run;
         else if (p.m_out) p.m_out[pend_row] = __float2half_rn(m_run);
       }
     }
-    if (ok && g > 0) ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j);
+    if (ok && g > 0) ok = epilogue(g - 1, pend_row, pend_l, pend_alpha, pend_rsum, pend_j, pend_kpow);
   }
   tc_fence_before();
   __syncthreads();

@@ -144,7 +144,7 @@ struct DecodeSpec {
 template <int D, int BC, bool SUMP = false, bool DEC = false>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                 int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream,
-                int l_from_p = 0, float* trace = nullptr, const DecodeSpec* dec = nullptr) {
+                int l_from_p = 0, float* trace = nullptr, const DecodeSpec* dec = nullptr, int two_level = 0) {
   using C = AttnCfg<D, BC>;
   const int Nk = dec ? dec->Nk : N;
   const uint64_t qrows = dec ? (uint64_t)B * Hkv * 128 : (uint64_t)B * Hq * N;
@@ -176,6 +176,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   p.inject = g_inject;
   p.l_from_p = l_from_p;
   p.trace = trace;
+  p.two_level = two_level;
   p.Nk = Nk;
   p.nq = dec ? dec->nq : 1;
   p.G = dec ? dec->G : 1;
@@ -189,6 +190,8 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
     p.causal = 0;
   }
   fill_neg_log2_scales(p.lneg);
+  p.lg2[0] = 0.0;
+  for (int i = 1; i < 16; ++i) p.lg2[i] = std::log2((double)i);
   // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM)
   static int per_sm = 0;
   if (per_sm == 0) {
@@ -209,7 +212,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
 template <bool SUMP>
 int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                   int N, int d, int causal, int kv_tile, void* o, void* m_out, void* l_out, int* status,
-                  cudaStream_t stream, int l_from_p, float* trace) {
+                  cudaStream_t stream, int l_from_p, float* trace, int two_level) {
   if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
@@ -223,7 +226,8 @@ int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qt
   if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
 #define HIFA4_LAUNCH(DD, BB) \
-  launch_attn<DD, BB, SUMP>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, l_from_p, trace)
+  launch_attn<DD, BB, SUMP>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, l_from_p, trace, \
+                            nullptr, two_level)
   if (d == 64) return kv_tile == 64 ? HIFA4_LAUNCH(64, 64) : HIFA4_LAUNCH(64, 128);
   if (d == 128) {
     if (kv_tile == 256) return HIFA4_LAUNCH(128, 256);
@@ -417,16 +421,17 @@ int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, con
                              int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
                              void* l_out, int* status, cudaStream_t stream) {
   return attn_dispatch<false>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream, 0,
-                              nullptr);
+                              nullptr, 0);
 }
 
 int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq,
-                            int Hkv, int N, int d, int causal, int kv_tile, int normaliser, float* trace, void* o,
-                            void* m_out, void* l_out, int* status, cudaStream_t stream) {
+                            int Hkv, int N, int d, int causal, int kv_tile, int normaliser, int two_level,
+                            float* trace, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
   if (normaliser != 0 && normaliser != 1) return HIFA4_ERR_INVALID_ARG;
+  if (two_level != 0 && two_level != 1) return HIFA4_ERR_INVALID_ARG;
   if (trace && !aligned16(trace)) return HIFA4_ERR_INVALID_ARG;
   return attn_dispatch<true>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream,
-                             normaliser, trace);
+                             normaliser, trace, two_level);
 }
 
 int hifa4_quantize_q_decode(const void* q, const int64_t q_strides[3], int B, int Hq, int Hkv, int nq, int d,

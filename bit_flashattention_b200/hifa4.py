@@ -53,7 +53,7 @@ def lib():
             "hifa4_rope_table": ([ctypes.c_double, i, i, i, P, P], i),
             "hifa4_quantize_qkv": ([P, P, P, P, P, P, i, i, i, i, i, P, P, QP, QP, QP, P, P], i),
             "hifa4_attn_fwd_quantized": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
-            "hifa4_attn_fwd_ablation": ([QP, QP, QP, i, i, i, i, i, i, i, i, P, P, P, P, P, P], i),
+            "hifa4_attn_fwd_ablation": ([QP, QP, QP, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P], i),
             "hifa4_quantize_q_decode": ([P, P, i, i, i, i, i, P, QP, P, P], i),
             "hifa4_decode_workspace_bytes": ([i, i, i, i], sz),
             "hifa4_attn_decode": ([QP, QP, QP, i, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
@@ -229,10 +229,11 @@ def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=
 
 
 def hifa4_attn_fwd_ablation(q: QTensor, k: QTensor, vt: QTensor, causal: bool, kv_tile: int = 0, normaliser: int = 0,
-                            trace=None, status=None, o=None, m=None, l=None):
+                            trace=None, status=None, o=None, m=None, l=None, two_level: bool = False):
     """Ablation form of the attention (see include/hifa4.h): normaliser 0 = HiFA4 (sum
-    P_hat), 1 = the inconsistent formulation (sum of unquantised P).  trace: optional fp32
-    [B, Hq, N, N/kv_tile, 2] receiving (sum P_hat, sum P) per (row, tile)."""
+    P_hat), 1 = the inconsistent formulation (sum of unquantised P); two_level selects the
+    two-level P scale (a per-row, per-tile power of two under the block scales of P).
+    trace: optional fp32 [B, Hq, N, N/kv_tile, 2] receiving (sum P_hat, sum P) per (row, tile)."""
     import torch
     dev = q.codes.device
     o = o if o is not None else torch.empty(q.B, q.H, q.N, q.d, dtype=torch.bfloat16, device=dev)
@@ -240,7 +241,8 @@ def hifa4_attn_fwd_ablation(q: QTensor, k: QTensor, vt: QTensor, causal: bool, k
     l = l if l is not None else torch.empty(q.B, q.H, q.N, dtype=torch.float16, device=dev)
     st = status if status is not None else new_status(dev)
     _check(lib().hifa4_attn_fwd_ablation(q.c(), k.c(), vt.c(), q.B, q.H, k.H, q.N, q.d, int(causal), int(kv_tile),
-                                         int(normaliser), _ptr(trace), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
+                                         int(normaliser), int(bool(two_level)), _ptr(trace), _ptr(o), _ptr(m), _ptr(l),
+                                         _ptr(st), _stream()),
            "hifa4_attn_fwd_ablation")
     return o, m, l
 

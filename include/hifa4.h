@@ -204,16 +204,25 @@ HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtens
  *                 (PV still uses P_hat), i.e. each tile's contribution to O is scaled by
  *                 sum P_hat / sum P.  With Q and K quantised without Smooth-QK (s = NULL)
  *                 this is the abstract's "direct HIF4 quantization" baseline.
+ *   two_level 0: the one-level block scales of P_hat (as hifa4_attn_fwd_quantized);
+ *   two_level 1: a second-level scale for P: per row and kv tile a power of two 2^k,
+ *                k = max(floor(log2 p_t) - 10, -40) with p_t the tile's largest block amax
+ *                of P; block scale E4M3_RN(RN(amax * RN(1/6)) * 2^-k), P_hat = code *
+ *                scale * 2^k, and the code rule's L(sigma) taken for the effective scale
+ *                scale * 2^k.  Equal to two_level 0 wherever every one-level block scale
+ *                is a normal E4M3 value; keeps the blocks one level flushes to zero
+ *                (amax <= 6 * 2^-10).  l is the FP16 recursion on sum P_hat computed by the
+ *                tensor core in fp32, which the wider scale range can round.
  * trace: device fp32 [B, Hq, N, N / kv_tile, 2] (16-byte aligned) or NULL; entry (row,
  *   tile, 0) = sum P_hat (exact), (row, tile, 1) = sum P of that tile, for every tile the
  *   row's 128-row query tile visits (causal: later tiles are not written; a visited tile
  *   with no visible key for the row holds 0, 0).  The per-tile mass error of the abstract
  *   is eps = sum P_hat / sum P - 1.
- * HIFA4_ERR_INVALID_ARG for normaliser outside {0, 1} or a misaligned trace.
+ * HIFA4_ERR_INVALID_ARG for normaliser or two_level outside {0, 1} or a misaligned trace.
  */
 HIFA4_API int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt,
                                       int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, int normaliser,
-                                      float* trace, void* o, void* m_out, void* l_out, int* status,
+                                      int two_level, float* trace, void* o, void* m_out, void* l_out, int* status,
                                       cudaStream_t stream);
 
 /*

@@ -2,7 +2,10 @@
 the HiFA4 normaliser reproduces the main kernel bit for bit; the per-(row, tile) trace of
 sum P_hat and sum P matches the oracle's tile loop; the inconsistent normaliser (l from
 the unquantised P) matches the oracle's l_from_p mode; and at full size the mean tile
-mass error eps = sum P_hat / sum P - 1 is negative (net mass loss, HiFA4 abstract)."""
+mass error eps = sum P_hat / sum P - 1 is negative (net mass loss, HiFA4 abstract).  The
+two-level P scale matches the oracle's two-level mode (m exact, l within one FP16 ulp, O
+within tolerance) and at full size keeps more of the mass and stays closer to exact
+attention than the one-level form, which itself beats direct 4-bit quantisation."""
 import numpy as np
 import pytest
 import torch
@@ -109,3 +112,112 @@ def test_full_size_mass_error_is_negative():
     print(f"\nqwen3-8b-4k full size: median eps-bar {med:.4f} over {ebar.numel()} tiles, "
           f"mean {float(ebar.mean()):.4f}, 5/95% {float(ebar.quantile(0.05)):.4f} / {float(ebar.quantile(0.95)):.4f}")
     assert med < 0.0
+
+
+def _check_two_level(w, qq, kq, vq, qz, rows=None):
+    nt = w.N // w.bc
+    trace = torch.full((w.B, w.Hq, w.N, nt, 2), -1.0, dtype=torch.float32, device="cuda")
+    st = hifa4.new_status("cuda")
+    o, m, l = hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=w.causal, kv_tile=w.bc, normaliser=0, trace=trace,
+                                            status=st, two_level=True)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    rows = np.arange(w.B * w.Hq * w.N, dtype=np.int64) if rows is None else rows
+    ref = oracle.attn_fwd(qz, w.causal, w.bc, rows, two_level=True)
+    mg = m.reshape(-1).float().cpu().numpy()[rows]
+    lg = l.reshape(-1).float().cpu().numpy()[rows]
+    assert np.array_equal(mg, ref["m"])
+    # sum P_hat of a tile spans a wider range of scales than one level: the tensor core's
+    # fp32 sum can round, so the fp16 l may split by one ulp
+    ulp = np.spacing(ref["l"].astype(np.float16)).astype(np.float64)
+    dl = np.abs(lg.astype(np.float64) - ref["l"])
+    assert np.all(dl <= ulp), float((dl / ulp).max())
+    assert np.mean(dl == 0) >= 0.99
+    stats = gc.compare_outputs(w, rows, o, m, l, ref)
+    assert stats["o_finite"] and stats["o_max_abs"] <= gc.O_MAX_ABS and stats["o_mean_rel"] <= gc.O_MEAN_REL, stats
+    tr = trace.reshape(-1, nt, 2).cpu().numpy()
+    for row in rows[:: max(1, len(rows) // 16)]:
+        t = oracle.attn_trace(qz, w.causal, w.bc, int(row), two_level=True)
+        visited = t["p"].shape[0]
+        sum_ph = t["phat"].astype(np.float64).sum(axis=1)
+        assert np.allclose(tr[row, :visited, 0], sum_ph, rtol=3e-5, atol=1e-30), row
+
+
+@pytest.mark.parametrize("name,kw", CASES)
+def test_two_level_matches_oracle(name, kw):
+    w = configs.scaled(configs.get(name), **kw)
+    qq, kq, vq, qz = _prepare(w)
+    _check_two_level(w, qq, kq, vq, qz)
+
+
+@pytest.mark.parametrize("d,bc", [(128, 256), (128, 128), (64, 64), (256, 64)])
+def test_two_level_on_score_spread_rows(d, bc):
+    # queries scaled up: rows span tens of log2 units, so most tiles have blocks below the
+    # one-level range and k changes from tile to tile (the O rescale by alpha * 2^(k_prev - k))
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=4, Hkv=2, N=1024, d=d, bc=bc)
+    q, k, v = gen.inputs(w)
+    qf = gen.bf16_bits_to_f32(q) * np.float32(3.0)
+    q = gen.f32_to_bf16_bits(qf.astype(np.float32))
+    qq, kq, vq, _ = gc.gpu_quantize(w, q, k, v, None, None)
+    qz = oracle.quantize_all(q, k, v)
+    rows = np.random.default_rng(9).choice(w.B * w.Hq * w.N, 512, replace=False).astype(np.int64)
+    _check_two_level(w, qq, kq, vq, qz, rows)
+    # and the two-level form differs from one level there (blocks one level flushes)
+    st = hifa4.new_status("cuda")
+    _, _, l1 = hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=w.causal, kv_tile=w.bc, status=st)
+    _, _, l2 = hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=w.causal, kv_tile=w.bc, status=st, two_level=True)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    assert float((l2.float() - l1.float()).mean()) > 0.0
+
+
+def _mean_tile_eps(w, qq, kq, vq, two_level):
+    nt = w.N // w.bc
+    trace = torch.zeros((w.B, w.Hq, w.N, nt, 2), dtype=torch.float32, device="cuda")
+    st = hifa4.new_status("cuda")
+    hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=w.causal, kv_tile=w.bc, normaliser=0, trace=trace, status=st,
+                                  two_level=two_level)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    tr = trace.reshape(w.B * w.Hq, w.N // 128, 128, nt, 2)
+    sp, sph = tr[..., 1].double(), tr[..., 0].double()
+    valid = sp > 0
+    eps = torch.where(valid, sph / torch.where(valid, sp, torch.ones_like(sp)) - 1.0, torch.zeros_like(sp))
+    n = valid.sum(dim=2)
+    return (eps.sum(dim=2) / n.clamp(min=1))[n > 0]
+
+
+def test_full_size_two_level_keeps_more_mass():
+    w = configs.get("qwen3-8b-4k")
+    qq, kq, vq, _ = _prepare(w)
+    e1 = _mean_tile_eps(w, qq, kq, vq, False)
+    e2 = _mean_tile_eps(w, qq, kq, vq, True)
+    print(f"\nqwen3-8b-4k full size eps-bar median / mean: one level {float(e1.median()):.4f} / "
+          f"{float(e1.mean()):.4f}, two-level {float(e2.median()):.4f} / {float(e2.mean()):.4f}")
+    assert abs(float(e2.median())) < abs(float(e1.median()))
+    assert abs(float(e2.mean())) < abs(float(e1.mean()))
+
+
+def test_full_size_error_against_exact_attention():
+    # relative error of the bf16 output against fp64 softmax attention of the bf16 inputs,
+    # on every 8th query row of every head: HiFA4 (Smooth-QK, consistent normaliser), its
+    # two-level P scale, and direct 4-bit quantisation (no smoothing, normaliser from P)
+    w = configs.get("qwen3-8b-4k")
+    q, k, v = gen.inputs(w)
+    s, sinv = gc.smooth_scales(w)
+    st = hifa4.new_status("cuda")
+    qq, kq, vq, _ = gc.gpu_quantize(w, q, k, v, s, sinv)
+    o1, _, _ = hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=True, kv_tile=w.bc, status=st)
+    o2, _, _ = hifa4.hifa4_attn_fwd_ablation(qq, kq, vq, causal=True, kv_tile=w.bc, status=st, two_level=True)
+    dq, dk, dv, _ = gc.gpu_quantize(w, q, k, v, None, None)
+    od, _, _ = hifa4.hifa4_attn_fwd_ablation(dq, dk, dv, causal=True, kv_tile=w.bc, normaliser=1, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    sel = torch.arange(0, w.N, 8, device="cuda")
+    qd = gc.bf16_dev(q).double()[:, :, sel]
+    kd = gc.bf16_dev(k).double().repeat_interleave(w.Hq // w.Hkv, dim=1)
+    vd = gc.bf16_dev(v).double().repeat_interleave(w.Hq // w.Hkv, dim=1)
+    S = qd @ kd.transpose(-1, -2) / np.sqrt(w.d)
+    S = S.masked_fill(torch.arange(w.N, device="cuda")[None, :] > sel[:, None], float("-inf"))
+    ref = torch.softmax(S, dim=-1) @ vd
+    rel = lambda o: float((o[:, :, sel].double() - ref).abs().mean() / ref.abs().mean())
+    e1, e2, ed = rel(o1), rel(o2), rel(od)
+    print(f"\nqwen3-8b-4k relative error vs fp64 attention: HiFA4 {e1:.4f}, two-level {e2:.4f}, direct 4-bit {ed:.4f}")
+    assert e1 < ed
+    assert e2 <= e1 * 1.02
