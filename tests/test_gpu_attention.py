@@ -4,6 +4,7 @@ synthetic inputs of every workload family (reduced sizes compared on every row; 
 sizes on sampled rows), plus the bounded-wait timeout path."""
 import numpy as np
 import pytest
+import torch
 
 from bit_flashattention_b200 import configs, gen, hifa4
 from tests import gpu_common as gc
@@ -115,3 +116,27 @@ def test_timeout_is_reported_and_context_survives():
     assert code == hifa4.ERR_TIMEOUT
     # the context is still usable and the next call is correct
     gc.assert_parity(gc.run_parity(w))
+
+
+@pytest.mark.parametrize("zero_q", [True, False])
+def test_maximum_length(zero_q):
+    # the longest supported sequence, N = 63488 (N * 1.03 < 65504 keeps the FP16 l finite),
+    # causal with 256-key tiles, on sampled rows including the last.  With Q = 0 every
+    # score is 0: P_hat = 1.03125 for every visible key, and the last row's FP16 l, summed
+    # tile by tile with one FP16 rounding each, ends just under the FP16 maximum
+    import oracle
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=1, Hkv=1, N=63488)
+    q, k, v = gen.inputs(w)
+    if zero_q:
+        q = np.zeros_like(q)
+    qq, kq, vq, vt = gc.gpu_quantize(w, q, k, v, None, None)
+    o, m, l, code = gc.gpu_attention(w, qq, kq, vt)
+    assert code == hifa4.OK, hifa4.status_string(code)
+    qz = oracle.quantize_all(q, k, v)
+    rows = np.array([0, 1, 255, 256, 31000, w.N - 257, w.N - 2, w.N - 1], np.int64)
+    ref = oracle.attn_fwd(qz, w.causal, w.bc, rows)
+    gc.assert_parity(gc.compare_outputs(w, rows, o, m, l, ref))
+    lg = l.reshape(-1).float()
+    assert bool(torch.isfinite(lg).all()) and float(lg.max()) < 65504.0
+    if zero_q:
+        assert float(lg[-1]) > 60000.0
