@@ -291,30 +291,57 @@ def run_gpu(args):
     if hifa4.hifa4_read_status(st) != hifa4.OK:
         raise RuntimeError("fused RoPE quantiser reported an error")
 
-    # e2e through the public API with host buffers: H2D of Q, K, V from pinned memory,
-    # the hot path, D2H of O, m, l -- every step
-    e2e_steps = max(3, min(args.steps, 20))
-    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    mh = torch.empty(m.shape, dtype=m.dtype, pin_memory=True)
-    lh = torch.empty(l.shape, dtype=l.dtype, pin_memory=True)
-    qd, kd, vd = sets[0]
+    # e2e through the public API with host buffers: every step copies its Q, K, V from
+    # pinned host memory, runs the hot path and reads O, m, l back to pinned host memory.
+    # As in a serving loop, the copies of neighbouring steps overlap the compute: H2D and
+    # D2H run on their own streams (one copy engine each way) into double-buffered device
+    # inputs and outputs, ordered by events.  The timed region spans the first H2D to the
+    # last D2H.
+    e2e_steps = max(4, min(args.steps, 20))
+    h2d_s = torch.cuda.Stream(device)
+    d2h_s = torch.cuda.Stream(device)
+    din = [sets[0], sets[1] if len(sets) > 1 else tuple(torch.empty_like(x) for x in sets[0])]
+    dout = [(o, m, l), tuple(torch.empty_like(x) for x in (o, m, l))]
+    hout = [tuple(torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in (o, m, l)) for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]         # step's inputs on the device
+    ev_in_free = [torch.cuda.Event() for _ in range(2)]    # quantiser done reading them
+    ev_out = [torch.cuda.Event() for _ in range(2)]        # step's outputs written
+    ev_out_free = [torch.cuda.Event() for _ in range(2)]   # outputs read back to the host
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(h2d_s)
     for i in range(e2e_steps):
-        qd.copy_(host[0], non_blocking=True)
-        kd.copy_(host[1], non_blocking=True)
-        vd.copy_(host[2], non_blocking=True)
-        step(0)
-        oh.copy_(o, non_blocking=True)
-        mh.copy_(m, non_blocking=True)
-        lh.copy_(l, non_blocking=True)
-    e1.record(stream)
+        j = i & 1
+        if i >= 2:
+            h2d_s.wait_event(ev_in_free[j])
+        with torch.cuda.stream(h2d_s):
+            for x, hx in zip(din[j], host):
+                x.copy_(hx, non_blocking=True)
+        ev_in[j].record(h2d_s)
+        stream.wait_event(ev_in[j])
+        if i >= 2:
+            stream.wait_event(ev_out_free[j])
+        qt, kt, vt = din[j]
+        hifa4.hifa4_quantize_qkv(qt, kt, vt, s, sinv, status=st, out=(qq[j], kq[j], vq[j]))
+        ev_in_free[j].record(stream)
+        ot, mt, lt = dout[j]
+        hifa4.hifa4_attn_fwd_quantized(qq[j], kq[j], vq[j], causal=w.causal, kv_tile=w.bc, status=st, o=ot, m=mt,
+                                       l=lt)
+        ev_out[j].record(stream)
+        d2h_s.wait_event(ev_out[j])
+        with torch.cuda.stream(d2h_s):
+            for hx, x in zip(hout[j], dout[j]):
+                hx.copy_(x, non_blocking=True)
+        ev_out_free[j].record(d2h_s)
+    e1.record(d2h_s)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    if hifa4.hifa4_read_status(st) != hifa4.OK:
+        raise RuntimeError("end-to-end steps reported an error")
+    oh, mh, lh = hout[0]
 
     elapsed = reduce_max(elapsed, dist, device)
     e2e_ms = reduce_max(e2e_ms, dist, device)
@@ -371,7 +398,9 @@ def run_gpu(args):
                      "algorithmic_bytes": attn_bytes,
                      "peak_source": f"{src} bf16 burst x {FP4_OVER_BF16:g} (nominal FP4/BF16 ratio)"},
         "e2e": {"value": round(e2e["tflops"], 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "note": "every step: H2D of Q, K, V from pinned memory, the hot path, D2H of O, m, l; the copies "
+                        "of neighbouring steps overlap the compute on their own streams (double-buffered)"},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }

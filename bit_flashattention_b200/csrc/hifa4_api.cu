@@ -91,11 +91,24 @@ int num_sms();
 // Grid of a grid-stride kernel: all units at once if they fit, else one full wave.
 template <typename K>
 int resident_grid(K kernel, int threads, int units) {
-  static int per_sm = 0;
-  if (per_sm == 0) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n <= 0) n = 1;
-    per_sm = n;
+  // kernels of one signature share K: cache the occupancy per kernel address
+  static std::mutex mu;
+  static const void* keys[16];
+  static int vals[16];
+  static int nkeys = 0;
+  int per_sm = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < nkeys; ++i)
+      if (keys[i] == reinterpret_cast<const void*>(kernel)) per_sm = vals[i];
+    if (per_sm == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm <= 0)
+        per_sm = 1;
+      if (nkeys < 16) {
+        keys[nkeys] = reinterpret_cast<const void*>(kernel);
+        vals[nkeys++] = per_sm;
+      }
+    }
   }
   const long long cap = (long long)per_sm * num_sms();
   return (int)(units < cap ? units : cap);
