@@ -88,44 +88,11 @@ __device__ __forceinline__ uint32_t encode8_pairs(const float2 (&y)[4]) {
   return w;
 }
 
-// max(a, |b|) that turns NaN into NaN (PTX max.NaN), so one test of a block's amax
-// catches every non-finite element of the block.
-__device__ __forceinline__ float max_abs_nan(float a, float b) {
-  float d;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(fabsf(b)));
-  return d;
-}
-
 // Scale code of a block from its absolute maximum, reciprocal from the table below.
 __device__ __forceinline__ uint32_t block_scale_tab(float amax, const float* rtab, float& R) {
   const uint32_t sc = cvt_e4m3(__fmul_rn(amax, kSixth));
   R = rtab[sc];
   return sc;
-}
-
-// Scale code and reciprocal of a block from its absolute maximum.
-__device__ __forceinline__ uint32_t block_scale(float amax, float& R) {
-  const uint32_t sc = cvt_e4m3(__fmul_rn(amax, kSixth));
-  const float sig = e4m3_value(sc);
-  R = (sig == 0.0f) ? 0.0f : __frcp_rn(sig);
-  return sc;
-}
-
-// Eight values -> eight E2M1 codes (after multiplying by R), packed low nibble first.
-__device__ __forceinline__ uint32_t encode8(const float (&x)[8], float R) {
-  float y[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) y[k] = __fmul_rn(x[k], R);
-  uint32_t w;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(w)
-      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
-  return w;
 }
 
 // RN(1/scale) for every E4M3 code (0 for the zero scale and for codes that are not
