@@ -221,6 +221,14 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   return cuda_status(cudaGetLastError());
 }
 
+// The kv tile chosen for kv_tile = 0: 256 keys at d = 128 when the key count allows it,
+// else 128; 128 at d = 64; 64 at d = 256.
+int default_kv_tile(int d, int nkeys) {
+  if (d == 256) return 64;
+  if (d == 128 && nkeys % 256 == 0) return 256;
+  return 128;
+}
+
 // Validation and dispatch shared by the plain and the ablation entry points.
 template <bool SUMP>
 int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
@@ -229,7 +237,7 @@ int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qt
   if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : (d == 128 ? 256 : 128);
+  if (kv_tile == 0) kv_tile = default_kv_tile(d, N);
   if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (d == 256 && kv_tile != 64) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (d == 64 && kv_tile == 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
@@ -478,7 +486,7 @@ int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || (Hq / Hkv) * nq > 128 || Nk <= 0 || Nk % 128 ||
       Nk > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (kv_tile == 0) kv_tile = (d == 256) ? 64 : (d == 128 ? 256 : 128);
+  if (kv_tile == 0) kv_tile = default_kv_tile(d, Nk);
   if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if ((d == 256 && kv_tile != 64) || (d == 64 && kv_tile == 256) || Nk % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q, B, Hkv, 128, d, 0) || !qt_ok(k, B, Hkv, Nk, d, 0) || !qt_ok(vt, B, Hkv, Nk, d, 1))

@@ -185,8 +185,9 @@ HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, co
  *   r      = P_hat * 1                           (4-bit MMA against ones: P-Reordering)
  *   l      = fp16_RN(fma(alpha, l, r)),  m = m_new
  * and finally out = bf16_RN(O / l).  kv_tile is 64, 128 or 256 and is part of the result's
- * definition; N must be a multiple of it.  0 selects 128 for d = 64, 256 for d = 128 and
- * 64 for d = 256; d = 256 supports only 64 and d = 64 at most 128.
+ * definition; N must be a multiple of it.  0 selects 128 for d = 64, 256 for d = 128 when
+ * N is a multiple of 256 (else 128), and 64 for d = 256; d = 256 supports only 64 and
+ * d = 64 at most 128.
  * o: bf16 [B, Hq, N, d] dense.  m_out, l_out: fp16 [B, Hq, N] dense, or NULL.
  */
 HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,

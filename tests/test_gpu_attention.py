@@ -140,3 +140,21 @@ def test_maximum_length(zero_q):
     assert bool(torch.isfinite(lg).all()) and float(lg.max()) < 65504.0
     if zero_q:
         assert float(lg[-1]) > 60000.0
+
+
+def test_default_kv_tile_when_n_is_not_a_multiple_of_256():
+    # d = 128 defaults to 256-key tiles; N = 384 is not a multiple of 256, so the default
+    # must fall back to 128-key tiles (and agree with the oracle at that tile)
+    import oracle
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=384, bc=128)
+    q, k, v = gen.inputs(w)
+    qq, kq, vq, _ = gc.gpu_quantize(w, q, k, v, None, None)
+    st = hifa4.new_status("cuda")
+    o0, m0, l0 = hifa4.hifa4_attn_fwd_quantized(qq, kq, vq, causal=True, kv_tile=0, status=st)
+    o1, m1, l1 = hifa4.hifa4_attn_fwd_quantized(qq, kq, vq, causal=True, kv_tile=128, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16)) and torch.equal(m0, m1) and torch.equal(l0, l1)
+    qz = oracle.quantize_all(q, k, v)
+    rows = np.arange(w.B * w.Hq * w.N, dtype=np.int64)
+    ref = oracle.attn_fwd(qz, True, 128, rows)
+    gc.assert_parity(gc.compare_outputs(w, rows, o0, m0, l0, ref))
