@@ -57,7 +57,6 @@ struct RowsUnit {
 template <int D, bool ROPE = false, bool PACK = false>
 __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit, const float* rtab, bool& bad) {
   using U = RowsUnit<D>;
-  const int lane = threadIdx.x & 31;
   const int blk = threadIdx.x % U::BPR;
   const int rsub = threadIdx.x / U::BPR;
   const int per_head = a.N / U::ROWS;
@@ -102,6 +101,7 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
       s2[2 * q + 1] = make_float2(t.z, t.w);
     }
   }
+  float nan_acc = 0.0f;                                // NaN / inf of any block amax survives the max
 #pragma unroll
   for (int k = 0; k < U::PASSES; ++k) {
     const int row = n0 + rsub + k * U::RPP;
@@ -140,7 +140,8 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     float amax = 0.0f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
-    bad |= !isfinite(amax);
+    if constexpr (ROPE) bad |= !isfinite(amax);              // (no register to spare across passes)
+    else nan_acc = max3_abs_nan(nan_acc, amax, amax);
     float R;
     const uint32_t sc = block_scale_tab(amax, rtab, R);
     const float2 R2 = make_float2(R, R);
@@ -149,14 +150,20 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
     *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
         make_uint2(encode8_pairs(lo), encode8_pairs(hi));
-    uint32_t word = sc << (8 * (lane & 3));
-    word |= __shfl_xor_sync(0xffffffffu, word, 1);
-    word |= __shfl_xor_sync(0xffffffffu, word, 2);
-    if ((lane & 3) == 0) {
-      uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
-      *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
+    uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
+    if constexpr (ROPE) {
+      // the four blocks of a 64-wide chunk (lanes 4q..4q+3) assemble the scale word
+      const int lane = threadIdx.x & 31;
+      uint32_t word = sc << (8 * (lane & 3));
+      word |= __shfl_xor_sync(0xffffffffu, word, 1);
+      word |= __shfl_xor_sync(0xffffffffu, word, 2);
+      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
+    } else {
+      // the block's scale byte: block (blk & 3) of its 64-wide chunk in the row's record
+      atom[sf_atom_offset(row % 128, blk & 3)] = (uint8_t)sc;
     }
   }
+  if constexpr (!ROPE) bad |= !isfinite(nan_acc);
 }
 
 // Grid-stride over Q units then K units.
