@@ -162,10 +162,13 @@ def measure_decode(hifa4, torch, device, steps, dist):
         del kb, vb
     del qdummy
     kv_bytes = 2 * B * Hkv * Nk * d * (0.5 + 1 / 16)
-    out = {"B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "Nk": Nk, "kv_tile": 256, "nsplit": "auto",
+    out = {"B": B, "Hq": Hq, "Hkv": Hkv, "d": d, "Nk": Nk, "kv_tile": "default", "nsplit": "auto",
            "kv_cache_bytes": kv_bytes}
     ws = None
-    for nq in (1, 32):
+    # nq = 1 and 32 at the default tile (nq = 1: 128-key tiles with the keys on the MMA's M
+    # dimension; nq = 32: 256-key tiles, 128 packed rows), and nq = 1 at 256-key tiles
+    # through the 128-row kernel for comparison
+    for name, nq, kv_tile in (("nq1", 1, 0), ("nq32", 32, 0), ("nq1_kv256", 1, 256)):
         q = torch.randn(B, Hq, nq, d, generator=gen_, device=device, dtype=torch.float32).to(torch.bfloat16)
         qp = hifa4.QTensor(B, Hkv, 128, d, 0, device)
         o = torch.empty(B, Hq, nq, d, dtype=torch.bfloat16, device=device)
@@ -174,7 +177,7 @@ def measure_decode(hifa4, torch, device, steps, dist):
 
         def dstep():
             hifa4.hifa4_quantize_q_decode(q, Hkv, status=st, out=qp)
-            hifa4.hifa4_attn_decode(qp, kq, vq, Hq, nq, kv_tile=256, nsplit=0, status=st, workspace=ws, o=o)
+            hifa4.hifa4_attn_decode(qp, kq, vq, Hq, nq, kv_tile=kv_tile, nsplit=0, status=st, workspace=ws, o=o)
 
         for _ in range(3):
             dstep()
@@ -190,9 +193,10 @@ def measure_decode(hifa4, torch, device, steps, dist):
             raise RuntimeError("decode reported an error")
         us = e0.elapsed_time(e1) / steps * 1e3
         us = reduce_max(us, dist, device)
-        out[f"nq{nq}"] = {"us_per_step": round(us, 2), "tokens_per_s": round(B * nq / (us * 1e-6), 1),
-                          "kv_gbs": round(kv_bytes / (us * 1e-6) / 1e9, 1),
-                          "attn_tflops": round(4.0 * B * Hq * nq * Nk * d / (us * 1e-6) / 1e12, 2)}
+        out[name] = {"kv_tile": kv_tile or (128 if nq == 1 else 256), "us_per_step": round(us, 2),
+                     "tokens_per_s": round(B * nq / (us * 1e-6), 1),
+                     "kv_gbs": round(kv_bytes / (us * 1e-6) / 1e9, 1),
+                     "attn_tflops": round(4.0 * B * Hq * nq * Nk * d / (us * 1e-6) / 1e12, 2)}
     out["note"] = ("step = packed-query quantiser + split attention + merge; kv_gbs = 4-bit K and V^T "
                    "(codes + scales) bytes / step time; the 0.6 GB cache exceeds L2")
     return out

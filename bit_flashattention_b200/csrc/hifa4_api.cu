@@ -11,6 +11,7 @@
 
 #include "../../include/hifa4.h"
 #include "attn.cuh"
+#include "attn_decode.cuh"
 #include "quant.cuh"
 
 using namespace hifa4;
@@ -218,6 +219,73 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   const long long cap = (long long)per_sm * num_sms();
   const unsigned grid = (unsigned)(units < cap ? units : cap);
   k_attn_fwd<D, BC, SUMP, DEC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+// Resident CTAs of the transposed decode kernel over the GPU.
+template <int NQ>
+int decode_t_resident() {
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    int n = 0;
+    if (!set_smem(k_attn_decode_t<NQ>, DecTCfg::SMEM) ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_decode_t<NQ>, DecTCfg::NTHREADS, DecTCfg::SMEM) !=
+            cudaSuccess ||
+        n <= 0)
+      n = 1;
+    if (n > (int)(512 / DecTCfg::TMEM_COLS)) n = 512 / DecTCfg::TMEM_COLS;
+    per_sm = n;
+  }
+  return per_sm * num_sms();
+}
+
+int decode_t_resident_for(int rows) {
+  return rows <= 4 ? decode_t_resident<4>() : (rows <= 8 ? decode_t_resident<8>() : decode_t_resident<16>());
+}
+
+// Decode with keys on the MMA's M dimension (k_attn_decode_t, head dim 128, 128-key tiles,
+// at most 16 packed query rows): NQ = the smallest of 4, 8, 16 that holds G * nq.  The
+// split count, when the caller leaves it open, is the one (of at most 16 and at least 16
+// tiles per split) whose units fill the resident CTAs' rounds best.
+template <int NQ>
+int launch_decode_t(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hkv,
+                    const DecodeSpec& dec, int* status, cudaStream_t stream) {
+  using C = DecTCfg;
+  constexpr int D = C::D;
+  const int Nk = dec.Nk;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q->codes, D / 2, (uint64_t)B * Hkv * 128, D / 2, D / 2, C::NMMA) ||
+      !make_map(&tk, k->codes, D / 2, (uint64_t)B * Hkv * Nk, D / 2, D / 2, C::BC) ||
+      !make_map(&tv, vt->codes, Nk / 2, (uint64_t)B * Hkv * D, Nk / 2, C::BC / 2, D))
+    return HIFA4_ERR_CUDA;
+  static bool attr = set_smem(k_attn_decode_t<NQ>, C::SMEM);
+  if (!attr) return HIFA4_ERR_CUDA;
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.qsf = static_cast<const uint8_t*>(q->scales);
+  p.ksf = static_cast<const uint8_t*>(k->scales);
+  p.vsf = static_cast<const uint8_t*>(vt->scales);
+  p.status = status;
+  p.B = B;
+  p.Hq = Hkv * dec.G;
+  p.Hkv = Hkv;
+  p.N = 128;
+  p.causal = 0;
+  p.c = (float)(1.4426950408889634074 / std::sqrt((double)D));
+  p.wait_ns = g_wait_ns;
+  p.Nk = Nk;
+  p.nq = dec.nq;
+  p.G = dec.G;
+  p.nsplit = dec.nsplit;
+  p.tps = dec.tps;
+  p.part_o = dec.part_o;
+  p.part_m = dec.part_m;
+  p.part_l = dec.part_l;
+  fill_neg_log2_scales(p.lneg);
+  const long long units = (long long)B * Hkv * dec.nsplit;
+  const long long cap = (long long)decode_t_resident<NQ>();
+  const unsigned grid = (unsigned)(units < cap ? units : cap);
+  k_attn_decode_t<NQ><<<grid, C::NTHREADS, C::SMEM, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -486,14 +554,32 @@ int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || nq <= 0 || (Hq / Hkv) * nq > 128 || Nk <= 0 || Nk % 128 ||
       Nk > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
-  if (kv_tile == 0) kv_tile = default_kv_tile(d, Nk);
+  const int rowsq = (Hq / Hkv) * nq;
+  // the transposed kernel: head dim 128, 128-key tiles, at most 16 packed query rows
+  const bool tpath = d == 128 && rowsq <= 16 && (kv_tile == 0 || kv_tile == 128);
+  if (kv_tile == 0) kv_tile = tpath ? 128 : default_kv_tile(d, Nk);
   if (kv_tile != 64 && kv_tile != 128 && kv_tile != 256) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if ((d == 256 && kv_tile != 64) || (d == 64 && kv_tile == 256) || Nk % kv_tile) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q, B, Hkv, 128, d, 0) || !qt_ok(k, B, Hkv, Nk, d, 0) || !qt_ok(vt, B, Hkv, Nk, d, 1))
     return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   const int ntile = Nk / kv_tile;
-  if (nsplit <= 0) {   // enough (batch, kv head, split) units for two waves over the SMs
+  if (nsplit <= 0 && tpath) {
+    // the split count (at most 16, at least 16 tiles per split) whose longest CTA path
+    // (rounds of resident CTAs x tiles per split) is closest to the even share
+    const long long res = decode_t_resident_for(rowsq), bk = (long long)B * Hkv;
+    const int maxs = ntile / 16 < 1 ? 1 : (ntile / 16 < 16 ? ntile / 16 : 16);
+    double best_eff = -1.0;
+    for (int ns = 1; ns <= maxs; ++ns) {
+      const int t = (ntile + ns - 1) / ns, nse = (ntile + t - 1) / t;
+      const long long rounds = (bk * nse + res - 1) / res;
+      const double eff = (double)bk * ntile / ((double)rounds * t * res);
+      if (eff > best_eff + 1e-9) {
+        best_eff = eff;
+        nsplit = ns;
+      }
+    }
+  } else if (nsplit <= 0) {   // enough (batch, kv head, split) units for two waves over the SMs
     const int want = (2 * num_sms() + B * Hkv - 1) / (B * Hkv);
     nsplit = want < 64 ? want : 64;
   }
@@ -507,9 +593,16 @@ int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa
   float* part_l = part_m + (size_t)B * Hkv * nsplit * 128;
   DecodeSpec spec{nq, Hq / Hkv, Nk, nsplit, tps, part_o, part_m, part_l};
   int rc;
+  if (tpath) {
+    rc = rowsq <= 4 ? launch_decode_t<4>(q, k, vt, B, Hkv, spec, status, stream)
+                    : (rowsq <= 8 ? launch_decode_t<8>(q, k, vt, B, Hkv, spec, status, stream)
+                                  : launch_decode_t<16>(q, k, vt, B, Hkv, spec, status, stream));
+    if (rc != HIFA4_OK) return rc;
+  }
 #define HIFA4_DEC(DD, BB) \
   launch_attn<DD, BB, false, true>(q, k, vt, B, Hq, Hkv, 128, 0, o, nullptr, nullptr, status, stream, 0, nullptr, &spec)
-  if (d == 64) rc = kv_tile == 64 ? HIFA4_DEC(64, 64) : HIFA4_DEC(64, 128);
+  if (tpath) rc = HIFA4_OK;
+  else if (d == 64) rc = kv_tile == 64 ? HIFA4_DEC(64, 64) : HIFA4_DEC(64, 128);
   else if (d == 128) rc = kv_tile == 256 ? HIFA4_DEC(128, 256) : (kv_tile == 64 ? HIFA4_DEC(128, 64) : HIFA4_DEC(128, 128));
   else rc = HIFA4_DEC(256, 64);
 #undef HIFA4_DEC

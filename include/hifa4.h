@@ -245,7 +245,10 @@ HIFA4_API int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtenso
  *     m = max m_s,  w_s = E(m_s - m) (0 for m_s = -inf),  L = fma(w_s, l_s, L),
  *     O = fma(w_s, O_s, O),  out = bf16_RN(O * RN(1/L)).
  *   o: bf16 [B, Hq, nq, d] dense; m_out, l_out: fp16 [B, Hq, nq] (m, RN(L)) or NULL.
- *   Nk a multiple of 128 and of kv_tile; kv_tile as for hifa4_attn_fwd_quantized.
+ *   Nk a multiple of 128 and of kv_tile; kv_tile as for hifa4_attn_fwd_quantized, except
+ *   that kv_tile = 0 selects 128 when d = 128 and G * nq <= 16.  That case (d = 128,
+ *   kv_tile = 128, G * nq <= 16) runs a kernel with the keys on the MMA's M dimension and
+ *   the packed query rows on N, with the same results as the 128-row kernel at that tile.
  */
 HIFA4_API int hifa4_quantize_q_decode(const void* q, const int64_t q_strides[3], int B, int Hq, int Hkv, int nq, int d,
                                       const float* s, const hifa4_qtensor* q_out, int* status, cudaStream_t stream);

@@ -20,6 +20,13 @@ CASES = [
     (64, 128, 4, 2, 3, 512, 2, False),
     (256, 64, 4, 2, 5, 384, 4, True),
     (128, 256, 4, 1, 16, 512, 1, False),      # one split: the merge is the identity
+    # keys on the MMA's M dimension (head dim 128, 128-key tiles, G * nq <= 16)
+    (128, 128, 32, 8, 1, 2048, 4, True),      # 4 query rows per kv head
+    (128, 0, 32, 8, 1, 2048, 3, True),        # the default tile is 128 keys here
+    (128, 128, 16, 2, 1, 1536, 5, False),     # 8 rows
+    (128, 128, 8, 2, 4, 1024, 3, True),       # 16 rows, the last tile masked per token
+    (128, 128, 4, 1, 3, 768, 2, False),       # 12 of 16 rows in use
+    (128, 128, 8, 1, 1, 512, 1, True),        # one split
 ]
 
 
@@ -64,7 +71,8 @@ def test_decode_matches_oracle(case):
     assert np.array_equal(_layout.rows_scales_to_plain(qp.scales.cpu().numpy(), B, Hkv, 128, d), qs)
     assert np.array_equal(kq.codes.cpu().numpy().reshape(kc.shape), kc)
 
-    ref = oracle.attn_decode(qc, qs, kc, ks, vc, vs, G=G, nq=nq, bc=kv_tile, nsplit=nsplit)
+    bc = kv_tile if kv_tile else 128
+    ref = oracle.attn_decode(qc, qs, kc, ks, vc, vs, G=G, nq=nq, bc=bc, nsplit=nsplit)
     mg = m.float().cpu().numpy()
     lg = l.float().cpu().numpy()
     assert np.array_equal(mg, ref["m"])
@@ -87,11 +95,13 @@ def _dequant_rows(codes, scales):
     return lut[nib] * np.repeat(sc, 16, axis=-1)
 
 
-def test_decode_error_does_not_grow_with_splits():
+@pytest.mark.parametrize("kv_tile", [256, 128])
+def test_decode_error_does_not_grow_with_splits(kv_tile):
     # different split counts quantise P_hat against different maxima: each count is a valid
     # evaluation, and its error against fp64 attention on the same dequantised operands stays
-    # at the single-split level; the automatic count must also run
-    case = (128, 256, 8, 2, 4, 4096, 1, False)
+    # at the single-split level; the automatic count must also run (128-key tiles: the
+    # kernel with keys on the MMA's M dimension)
+    case = (128, kv_tile, 8, 2, 4, 4096, 1, False)
     d, kv_tile, Hq, Hkv, nq, Nk, _, _ = case
     B, G = 2, Hq // Hkv
     q, k, v, _, _ = _case(*case)
