@@ -421,25 +421,37 @@ __global__ void __launch_bounds__(DecTCfg::NTHREADS, NQ == 16 ? 2 : 3)
           }
         }
         // P_hat^T: per query row q the 16-key block of this lane (lanes 0-15 / 16-31); even
-        // lanes pack the codes of keys k, k + 1 into one byte
+        // lanes pack the codes of keys k, k + 1 into one byte.  Each step runs over all rows
+        // before the next, so the rows' dependency chains overlap.
         uint8_t* pbuf = sP(pb);
         uint8_t* patom = sPsf(pb) + 512 * (b8 >> 2);
+        float bm[NQ];
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) bm[q] = s[q];
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) bm[q] = fmaxf(bm[q], __shfl_xor_sync(0xffffffffu, bm[q], off));
+        }
+        float y[NQ];
+        uint32_t sc[NQ];
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          float bm = s[q];
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-          bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-          const float pmax = exp2_own(__fmaf_rn(bm, c, -mnew[q]));
-          const uint32_t sc = cvt_e4m3(__fmul_rn(pmax, kSixth));
+          const float pmax = exp2_own(__fmaf_rn(bm[q], c, -mnew[q]));
+          sc[q] = cvt_e4m3(__fmul_rn(pmax, kSixth));
+        }
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
           // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-          const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew[q]), 125.0f), 0.0078125f);
+          const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc[q]], mnew[q]), 125.0f), 0.0078125f);
           const float v = __fmaf_rn(fma_sat(s[q], c7, B), 128.0f, kPhatM);
-          const float y = __uint_as_float(__float_as_uint(v) << 13);
-          const float yn = __shfl_xor_sync(0xffffffffu, y, 1);   // the next key's value
-          if ((lane & 1) == 0) pbuf[swz_offset(q, q4, C::PROW) + (lane >> 1)] = (uint8_t)cvt_e2m1x2(yn, y);
-          if ((lane & 15) == 0) patom[sf_atom_offset(q, b8 & 3)] = (uint8_t)sc;
+          y[q] = __uint_as_float(__float_as_uint(v) << 13);
+        }
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const float yn = __shfl_xor_sync(0xffffffffu, y[q], 1);   // the next key's value
+          if ((lane & 1) == 0) pbuf[swz_offset(q, q4, C::PROW) + (lane >> 1)] = (uint8_t)cvt_e2m1x2(yn, y[q]);
+          if ((lane & 15) == 0) patom[sf_atom_offset(q, b8 & 3)] = (uint8_t)sc[q];
         }
         fence_proxy_async_smem();
         if (jj > 0) {

@@ -227,12 +227,30 @@ template <int NQ>
 int decode_t_resident() {
   static int per_sm = 0;
   if (per_sm == 0) {
+    // several CTAs share an SM: the largest shared-memory carveout, and the count from the
+    // SM's shared memory, registers, threads and TMEM (the occupancy query can report
+    // fewer; a CTA beyond what fits only waits for a free slot)
     int n = 0;
-    if (!set_smem(k_attn_decode_t<NQ>, DecTCfg::SMEM) ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_decode_t<NQ>, DecTCfg::NTHREADS, DecTCfg::SMEM) !=
-            cudaSuccess ||
-        n <= 0)
-      n = 1;
+    set_smem(k_attn_decode_t<NQ>, DecTCfg::SMEM);
+    cudaFuncSetAttribute(k_attn_decode_t<NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_decode_t<NQ>, DecTCfg::NTHREADS, DecTCfg::SMEM) !=
+        cudaSuccess)
+      n = 0;
+    int dev = 0, smem_sm = 0, reserved = 0;
+    cudaFuncAttributes fa;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
+        cudaFuncGetAttributes(&fa, k_attn_decode_t<NQ>) == cudaSuccess && fa.numRegs > 0) {
+      const int by_smem = smem_sm / ((int)DecTCfg::SMEM + reserved);
+      const int by_regs = 65536 / (((fa.numRegs + 7) / 8 * 8) * DecTCfg::NTHREADS);
+      const int by_threads = 2048 / DecTCfg::NTHREADS;
+      int m = by_smem < by_regs ? by_smem : by_regs;
+      m = m < by_threads ? m : by_threads;
+      if (m > n) n = m;
+    }
+    if (n <= 0) n = 1;
     if (n > (int)(512 / DecTCfg::TMEM_COLS)) n = 512 / DecTCfg::TMEM_COLS;
     per_sm = n;
   }
