@@ -19,8 +19,11 @@
 // +31 of S^T, channels 32 (w & 3) .. +31 of O^T).  Per tile a softmax warp takes the
 // column maxima of its 32 keys with one integer max-reduction per query row, combines
 // the four warps' maxima through shared memory, forms the 16-key block maxima with four
-// shuffles, and packs the codes of neighbouring keys into bytes of the P_hat^T operand.
-// Every wait is bounded, as in k_attn_fwd.
+// shuffle rounds, and packs the codes of neighbouring keys into bytes of the P_hat^T
+// operand; each of these steps runs over all NQ rows before the next, so the rows'
+// dependency chains overlap.  With so little work per tile, latency is hidden by running
+// three CTAs per SM (73 KB of shared memory and 128 TMEM columns each).  Every wait is
+// bounded, as in k_attn_fwd.
 #pragma once
 #include "attn.cuh"
 
