@@ -155,6 +155,28 @@ struct DecodeSpec {
   float *part_o, *part_m, *part_l;
 };
 
+// CTAs of `kernel` that fit on one SM by its shared memory (dynamic `smem` plus static
+// and the per-block reservation), registers (per SM sub-partition: warps are spread over
+// four) and threads; 0 when the attributes cannot be read.
+template <typename K>
+int resident_by_limits(K kernel, int threads, int smem) {
+  int dev = 0, smem_sm = 0, reserved = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs <= 0)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int regs = (fa.numRegs + 7) / 8 * 8;
+  const int by_smem = smem_sm / (smem + (int)fa.sharedSizeBytes + reserved);
+  int by_regs = 0;   // CTAs whose warps, dealt round-robin over the 4 sub-partitions, fit 16384 registers each
+  while ((((by_regs + 1) * warps + 3) / 4) * 32 * regs <= 16384) ++by_regs;
+  const int by_threads = 2048 / threads;
+  int m = by_smem < by_regs ? by_smem : by_regs;
+  return m < by_threads ? m : by_threads;
+}
+
 template <int D, int BC, bool SUMP = false, bool DEC = false>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                 int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream,
@@ -210,9 +232,13 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   static int per_sm = 0;
   if (per_sm == 0) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem) != cudaSuccess ||
-        n <= 0)
-      n = 1;
+    cudaFuncSetAttribute(k_attn_fwd<D, BC, SUMP, DEC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem) != cudaSuccess)
+      n = 0;
+    const int m = resident_by_limits(k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem);
+    if (m > n) n = m;
+    if (n <= 0) n = 1;
     per_sm = n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
   }
   const long long units = dec ? (long long)B * Hkv * dec->nsplit : (long long)B * Hq * (N / 128);
@@ -228,8 +254,7 @@ int decode_t_resident() {
   static int per_sm = 0;
   if (per_sm == 0) {
     // several CTAs share an SM: the largest shared-memory carveout, and the count from the
-    // SM's shared memory, registers, threads and TMEM (the occupancy query can report
-    // fewer; a CTA beyond what fits only waits for a free slot)
+    // SM's limits (the occupancy query can report fewer)
     int n = 0;
     set_smem(k_attn_decode_t<NQ>, DecTCfg::SMEM);
     cudaFuncSetAttribute(k_attn_decode_t<NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -237,19 +262,8 @@ int decode_t_resident() {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_decode_t<NQ>, DecTCfg::NTHREADS, DecTCfg::SMEM) !=
         cudaSuccess)
       n = 0;
-    int dev = 0, smem_sm = 0, reserved = 0;
-    cudaFuncAttributes fa;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) == cudaSuccess &&
-        cudaFuncGetAttributes(&fa, k_attn_decode_t<NQ>) == cudaSuccess && fa.numRegs > 0) {
-      const int by_smem = smem_sm / ((int)DecTCfg::SMEM + reserved);
-      const int by_regs = 65536 / (((fa.numRegs + 7) / 8 * 8) * DecTCfg::NTHREADS);
-      const int by_threads = 2048 / DecTCfg::NTHREADS;
-      int m = by_smem < by_regs ? by_smem : by_regs;
-      m = m < by_threads ? m : by_threads;
-      if (m > n) n = m;
-    }
+    const int m = resident_by_limits(k_attn_decode_t<NQ>, DecTCfg::NTHREADS, DecTCfg::SMEM);
+    if (m > n) n = m;
     if (n <= 0) n = 1;
     if (n > (int)(512 / DecTCfg::TMEM_COLS)) n = 512 / DecTCfg::TMEM_COLS;
     per_sm = n;

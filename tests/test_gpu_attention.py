@@ -49,6 +49,7 @@ EDGE = [
     ("qwen3-8b-4k", dict(Hq=4, Hkv=4, N=512)),                         # no GQA
     ("llama3.1-8b-b4-16k", dict(B=3, Hq=2, Hkv=2, N=512, causal=False)),
     ("gemma2-9b-8k", dict(B=2, Hq=2, Hkv=1, N=128)),                   # d = 256, two 64-key tiles
+    ("qwen3-8b-4k", dict(B=2, Hq=4, Hkv=2, N=768, bc=64)),             # d = 128, 64-key tiles: two CTAs per SM
 ]
 
 
