@@ -90,6 +90,28 @@ bool d_ok(int d) { return d == 64 || d == 128 || d == 256; }
 int num_sms();
 
 // Grid of a grid-stride kernel: all units at once if they fit, else one full wave.
+// CTAs of `kernel` that fit on one SM by its shared memory (dynamic `smem` plus static
+// and the per-block reservation), registers (per SM sub-partition: warps are spread over
+// four) and threads; 0 when the attributes cannot be read.
+template <typename K>
+int resident_by_limits(K kernel, int threads, int smem) {
+  int dev = 0, smem_sm = 0, reserved = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs <= 0)
+    return 0;
+  const int warps = (threads + 31) / 32;
+  const int regs = (fa.numRegs + 7) / 8 * 8;
+  const int by_smem = smem_sm / (smem + (int)fa.sharedSizeBytes + reserved);
+  int by_regs = 0;   // CTAs whose warps, dealt round-robin over the 4 sub-partitions, fit 16384 registers each
+  while ((((by_regs + 1) * warps + 3) / 4) * 32 * regs <= 16384) ++by_regs;
+  const int by_threads = 2048 / threads;
+  int m = by_smem < by_regs ? by_smem : by_regs;
+  return m < by_threads ? m : by_threads;
+}
+
 template <typename K>
 int resident_grid(K kernel, int threads, int units) {
   // kernels of one signature share K: cache the occupancy per kernel address
@@ -103,8 +125,10 @@ int resident_grid(K kernel, int threads, int units) {
     for (int i = 0; i < nkeys; ++i)
       if (keys[i] == reinterpret_cast<const void*>(kernel)) per_sm = vals[i];
     if (per_sm == 0) {
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess || per_sm <= 0)
-        per_sm = 1;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess) per_sm = 0;
+      const int m = resident_by_limits(kernel, threads, 0);
+      if (m > per_sm) per_sm = m;
+      if (per_sm <= 0) per_sm = 1;
       if (nkeys < 16) {
         keys[nkeys] = reinterpret_cast<const void*>(kernel);
         vals[nkeys++] = per_sm;
@@ -154,28 +178,6 @@ struct DecodeSpec {
   int nq, G, Nk, nsplit, tps;
   float *part_o, *part_m, *part_l;
 };
-
-// CTAs of `kernel` that fit on one SM by its shared memory (dynamic `smem` plus static
-// and the per-block reservation), registers (per SM sub-partition: warps are spread over
-// four) and threads; 0 when the attributes cannot be read.
-template <typename K>
-int resident_by_limits(K kernel, int threads, int smem) {
-  int dev = 0, smem_sm = 0, reserved = 0;
-  cudaFuncAttributes fa;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
-      cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs <= 0)
-    return 0;
-  const int warps = (threads + 31) / 32;
-  const int regs = (fa.numRegs + 7) / 8 * 8;
-  const int by_smem = smem_sm / (smem + (int)fa.sharedSizeBytes + reserved);
-  int by_regs = 0;   // CTAs whose warps, dealt round-robin over the 4 sub-partitions, fit 16384 registers each
-  while ((((by_regs + 1) * warps + 3) / 4) * 32 * regs <= 16384) ++by_regs;
-  const int by_threads = 2048 / threads;
-  int m = by_smem < by_regs ? by_smem : by_regs;
-  return m < by_threads ? m : by_threads;
-}
 
 template <int D, int BC, bool SUMP = false, bool DEC = false>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,

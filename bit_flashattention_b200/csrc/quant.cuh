@@ -42,19 +42,13 @@ struct RowsUnit {
 // One unit (ROWS rows of one head) of the Q/K quantiser with 256 threads.  Thread
 // (row r, block k) quantises one 16-element block: two 16-byte loads (all of a thread's
 // loads in flight before any arithmetic), the block amax with 3-input max instructions,
-// the scale from the amax and its reciprocal from a shared table, 8 code bytes stored at
-// once.  The four blocks of a 64-wide chunk sit in lanes 4q..4q+3, which assemble the
-// chunk's scale word with two shuffles.
-//
-// ROPE: the rows are pre-RoPE; each thread also loads the partner block of its rotate-half
-// pair (channel c pairs with c +- D/2) and the angle table row of its token, and rotates
-// in fp32 with each product and sum rounded once:
-//   x'_c = RN(RN(x_c cos) - RN(x_{c+D/2} sin)),  x'_{c+D/2} = RN(RN(x_{c+D/2} cos) + RN(x_c sin)),
-// before Smooth-QK (which the HiFA4 abstract applies after RoPE).
+// the scale from the amax and its reciprocal from a shared table, 8 code bytes and the
+// scale byte stored directly; one NaN-propagating maximum per thread carries the
+// non-finite check.
 //
 // PACK: the unit is the 128-row decode tile of kv head h (H = Hkv): row r < G * nq is token
 // r % nq of query head h * G + r / nq of the [B, Hq, nq, D] input, rows >= G * nq are zero.
-template <int D, bool ROPE = false, bool PACK = false>
+template <int D, bool PACK = false>
 __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit, const float* rtab, bool& bad) {
   using U = RowsUnit<D>;
   const int blk = threadIdx.x % U::BPR;
@@ -63,10 +57,7 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
   const int bh = unit / per_head, n0 = (unit % per_head) * U::ROWS;
   const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
   const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + blk * 16;
-  constexpr int HB = U::BPR / 2;                      // blocks per half row
-  const bool first_half = blk < HB;
   uint4 raw[U::PASSES][2];
-  uint4 praw[ROPE ? U::PASSES : 1][2];
 #pragma unroll
   for (int k = 0; k < U::PASSES; ++k) {
     const int rr = n0 + rsub + k * U::RPP;
@@ -85,11 +76,6 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     const uint4* src = reinterpret_cast<const uint4*>(base + (long long)rr * a.sn);
     raw[k][0] = src[0];
     raw[k][1] = src[1];
-    if constexpr (ROPE) {
-      const uint4* ps = src + (first_half ? 2 * HB : -2 * HB);   // the partner block, D/2 channels away
-      praw[k][0] = ps[0];
-      praw[k][1] = ps[1];
-    }
   }
   float2 s2[8];
   if (a.scale) {
@@ -109,30 +95,6 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     float2 v[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
-    if constexpr (ROPE) {
-      const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&praw[k][0]);
-      const int tc = (blk % HB) * 16;                   // table column of the block's first channel
-      const float4* cp = reinterpret_cast<const float4*>(a.rope_cos + (long long)row * (D / 2) + tc);
-      const float4* sp = reinterpret_cast<const float4*>(a.rope_sin + (long long)row * (D / 2) + tc);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 c4 = __ldg(cp + q), s4 = __ldg(sp + q);
-        const float2 cs[2] = {make_float2(c4.x, c4.y), make_float2(c4.z, c4.w)};
-        const float2 sn[2] = {make_float2(s4.x, s4.y), make_float2(s4.z, s4.w)};
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          // scalar intrinsics: each product is rounded before the sum (never contracted into
-          // an fma, which would turn an exact cancellation into a signed rounding residue)
-          const int e = 2 * q + t;
-          const float2 y = __bfloat1622float2(q2[e]);
-          const float2 cc = cs[t], ss = sn[t];
-          const float ax = __fmul_rn(v[e].x, cc.x), ay = __fmul_rn(v[e].y, cc.y);
-          const float bx = __fmul_rn(y.x, ss.x), by = __fmul_rn(y.y, ss.y);
-          v[e] = first_half ? make_float2(__fsub_rn(ax, bx), __fsub_rn(ay, by))
-                            : make_float2(__fadd_rn(ax, bx), __fadd_rn(ay, by));
-        }
-      }
-    }
     if (a.scale) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], s2[e]);
@@ -140,8 +102,7 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     float amax = 0.0f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
-    if constexpr (ROPE) bad |= !isfinite(amax);              // (no register to spare across passes)
-    else nan_acc = max3_abs_nan(nan_acc, amax, amax);
+    nan_acc = max3_abs_nan(nan_acc, amax, amax);
     float R;
     const uint32_t sc = block_scale_tab(amax, rtab, R);
     const float2 R2 = make_float2(R, R);
@@ -150,20 +111,102 @@ __device__ __forceinline__ void quant_rows_unit(const QuantRowsArgs& a, int unit
     const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
     *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
         make_uint2(encode8_pairs(lo), encode8_pairs(hi));
+    // the block's scale byte: block (blk & 3) of its 64-wide chunk in the row's record
     uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
-    if constexpr (ROPE) {
-      // the four blocks of a 64-wide chunk (lanes 4q..4q+3) assemble the scale word
-      const int lane = threadIdx.x & 31;
-      uint32_t word = sc << (8 * (lane & 3));
-      word |= __shfl_xor_sync(0xffffffffu, word, 1);
-      word |= __shfl_xor_sync(0xffffffffu, word, 2);
-      if ((lane & 3) == 0) *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(row % 128, 0)) = word;
-    } else {
-      // the block's scale byte: block (blk & 3) of its 64-wide chunk in the row's record
-      atom[sf_atom_offset(row % 128, blk & 3)] = (uint8_t)sc;
+    atom[sf_atom_offset(row % 128, blk & 3)] = (uint8_t)sc;
+  }
+  bad |= !isfinite(nan_acc);
+}
+
+// Smooth-QK (when a.scale), amax, scale and codes of one 16-element block (row `row` of
+// head bh, block blk, values v): 8 code bytes and the scale byte (block blk & 3 of its
+// 64-wide chunk in the row's atom record).  nan_acc carries a NaN or infinity of any amax.
+template <int D>
+__device__ __forceinline__ void quant_block16(const QuantRowsArgs& a, int bh, int g, int row, int blk, float2 (&v)[8],
+                                              const float* rtab, float& nan_acc) {
+  if (a.scale) {
+    const float4* sp = reinterpret_cast<const float4*>(a.scale + g * D + blk * 16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 t = __ldg(sp + q);
+      v[2 * q] = __fmul2_rn(v[2 * q], make_float2(t.x, t.y));
+      v[2 * q + 1] = __fmul2_rn(v[2 * q + 1], make_float2(t.z, t.w));
     }
   }
-  if constexpr (!ROPE) bad |= !isfinite(nan_acc);
+  float amax = 0.0f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) amax = max3_abs_nan(amax, v[e].x, v[e].y);
+  nan_acc = max3_abs_nan(nan_acc, amax, amax);
+  float R;
+  const uint32_t sc = block_scale_tab(amax, rtab, R);
+  const float2 R2 = make_float2(R, R);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = __fmul2_rn(v[e], R2);
+  const float2 lo[4] = {v[0], v[1], v[2], v[3]}, hi[4] = {v[4], v[5], v[6], v[7]};
+  *reinterpret_cast<uint2*>(a.codes + ((long long)bh * a.N + row) * (D / 2) + blk * 8) =
+      make_uint2(encode8_pairs(lo), encode8_pairs(hi));
+  uint8_t* atom = a.sf + (((long long)bh * (a.N / 128) + row / 128) * (D / 64) + blk / 4) * 512;
+  atom[sf_atom_offset(row % 128, blk & 3)] = (uint8_t)sc;
+}
+
+// Fused RoPE unit (ROWS rows of one head, pre-RoPE input) with one thread per
+// rotate-half block pair: thread (row r, pair p) loads blocks p and p + D/32 of its row
+// (channels c and c + D/2 pair up element by element) and the pair's 16 angle-table
+// columns once, rotates in fp32 with every product and sum rounded once,
+//   x'_c = RN(RN(x_c cos) - RN(x_{c+D/2} sin)),  x'_{c+D/2} = RN(RN(x_{c+D/2} cos) + RN(x_c sin)),
+// then applies Smooth-QK and quantises both blocks.
+template <int D>
+struct RopeUnit {
+  static constexpr int HB = D / 32;                   // block pairs per row
+  static constexpr int RPP = 256 / HB;                // rows per pass
+  static constexpr int ROWS = RowsUnit<D>::ROWS;      // rows per unit (the host's unit count)
+  static constexpr int PASSES = ROWS / RPP;
+};
+
+template <int D>
+__device__ __forceinline__ void quant_rows_rope_pair(const QuantRowsArgs& a, int unit, const float* rtab, bool& bad) {
+  using U = RopeUnit<D>;
+  const int pr = threadIdx.x % U::HB, rsub = threadIdx.x / U::HB;
+  const int per_head = a.N / U::ROWS;
+  const int bh = unit / per_head, n0 = (unit % per_head) * U::ROWS;
+  const int b = bh / a.H, h = bh % a.H, g = h / (a.H / a.Hkv);
+  const __nv_bfloat16* base = a.x + b * a.sb + h * a.sh + pr * 16;
+  float nan_acc = 0.0f;
+#pragma unroll
+  for (int k = 0; k < U::PASSES; ++k) {
+    const int row = n0 + rsub + k * U::RPP;
+    const uint4* src = reinterpret_cast<const uint4*>(base + (long long)row * a.sn);
+    uint4 x1[2], x2[2];
+    x1[0] = src[0];
+    x1[1] = src[1];
+    x2[0] = src[2 * U::HB];                           // the partner block, D/2 channels on
+    x2[1] = src[2 * U::HB + 1];
+    const float4* cp = reinterpret_cast<const float4*>(a.rope_cos + (long long)row * (D / 2) + pr * 16);
+    const float4* sp = reinterpret_cast<const float4*>(a.rope_sin + (long long)row * (D / 2) + pr * 16);
+    float4 c4[4], s4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      c4[q] = __ldg(cp + q);
+      s4[q] = __ldg(sp + q);
+    }
+    const __nv_bfloat162* p1 = reinterpret_cast<const __nv_bfloat162*>(&x1[0]);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&x2[0]);
+    float2 v1[8], v2[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 a1 = __bfloat1622float2(p1[e]), a2 = __bfloat1622float2(p2[e]);
+      const float2 cc = (e & 1) ? make_float2(c4[e >> 1].z, c4[e >> 1].w) : make_float2(c4[e >> 1].x, c4[e >> 1].y);
+      const float2 ss = (e & 1) ? make_float2(s4[e >> 1].z, s4[e >> 1].w) : make_float2(s4[e >> 1].x, s4[e >> 1].y);
+      // scalar intrinsics: each product is rounded before the sum (never contracted)
+      v1[e] = make_float2(__fsub_rn(__fmul_rn(a1.x, cc.x), __fmul_rn(a2.x, ss.x)),
+                          __fsub_rn(__fmul_rn(a1.y, cc.y), __fmul_rn(a2.y, ss.y)));
+      v2[e] = make_float2(__fadd_rn(__fmul_rn(a2.x, cc.x), __fmul_rn(a1.x, ss.x)),
+                          __fadd_rn(__fmul_rn(a2.y, cc.y), __fmul_rn(a1.y, ss.y)));
+    }
+    quant_block16<D>(a, bh, g, row, pr, v1, rtab, nan_acc);
+    quant_block16<D>(a, bh, g, row, pr + U::HB, v2, rtab, nan_acc);
+  }
+  bad |= !isfinite(nan_acc);
 }
 
 // Grid-stride over Q units then K units.
@@ -187,7 +230,7 @@ __global__ void __launch_bounds__(256) k_quant_q_decode(QuantRowsArgs qa, int* s
   fill_recip_table(rtab, threadIdx.x, 256);
   __syncthreads();
   bool bad = false;
-  for (int u = blockIdx.x; u < qa.units; u += gridDim.x) quant_rows_unit<D, false, true>(qa, u, rtab, bad);
+  for (int u = blockIdx.x; u < qa.units; u += gridDim.x) quant_rows_unit<D, true>(qa, u, rtab, bad);
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }
 
@@ -200,8 +243,8 @@ __global__ void __launch_bounds__(256, 2) k_quant_rows_rope(QuantRowsArgs qa, Qu
   __syncthreads();
   bool bad = false;
   for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
-    if (u < qa.units) quant_rows_unit<D, true>(qa, u, rtab, bad);
-    else quant_rows_unit<D, true>(ka, u - qa.units, rtab, bad);
+    if (u < qa.units) quant_rows_rope_pair<D>(qa, u, rtab, bad);
+    else quant_rows_rope_pair<D>(ka, u - qa.units, rtab, bad);
   }
   if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }
