@@ -27,6 +27,8 @@ CASES = [
     (128, 128, 8, 2, 4, 1024, 3, True),       # 16 rows, the last tile masked per token
     (128, 128, 4, 1, 3, 768, 2, False),       # 12 of 16 rows in use
     (128, 128, 8, 1, 1, 512, 1, True),        # one split
+    (128, 0, 4, 1, 1, 128, 4, False),         # a single 128-key tile: more splits asked than tiles
+    (128, 128, 16, 1, 1, 384, 2, True),       # 16 query heads per kv head, one token each
 ]
 
 
