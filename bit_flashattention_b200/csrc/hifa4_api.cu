@@ -197,6 +197,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   static bool attr = set_smem(k_attn_fwd<D, BC, SUMP, DEC>, smem);
   if (!attr) return HIFA4_ERR_CUDA;
   AttnParams p;
+  std::memset(&p, 0, sizeof(p));
   p.qsf = static_cast<const uint8_t*>(q->scales);
   p.ksf = static_cast<const uint8_t*>(k->scales);
   p.vsf = static_cast<const uint8_t*>(vt->scales);
@@ -230,9 +231,9 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   fill_neg_log2_scales(p.lneg);
   p.lg2[0] = 0.0;
   for (int i = 1; i < 16; ++i) p.lg2[i] = std::log2((double)i);
-  // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM)
-  static int per_sm = 0;
-  if (per_sm == 0) {
+  // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM);
+  // computed once per kernel instance (a function-local static: thread-safe initialisation)
+  static const int per_sm = [smem] {
     int n = 0;
     cudaFuncSetAttribute(k_attn_fwd<D, BC, SUMP, DEC>, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
@@ -241,8 +242,8 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
     const int m = resident_by_limits(k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem);
     if (m > n) n = m;
     if (n <= 0) n = 1;
-    per_sm = n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
-  }
+    return n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
+  }();
   const long long units = dec ? (long long)B * Hkv * dec->nsplit : (long long)B * Hq * (N / 128);
   const long long cap = (long long)per_sm * num_sms();
   const unsigned grid = (unsigned)(units < cap ? units : cap);
@@ -253,8 +254,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
 // Resident CTAs of the transposed decode kernel over the GPU.
 template <int NQ>
 int decode_t_resident() {
-  static int per_sm = 0;
-  if (per_sm == 0) {
+  static const int per_sm = [] {
     // several CTAs share an SM: the largest shared-memory carveout, and the count from the
     // SM's limits (the occupancy query can report fewer)
     int n = 0;
@@ -268,8 +268,8 @@ int decode_t_resident() {
     if (m > n) n = m;
     if (n <= 0) n = 1;
     if (n > (int)(512 / DecTCfg::TMEM_COLS)) n = 512 / DecTCfg::TMEM_COLS;
-    per_sm = n;
-  }
+    return n;
+  }();
   return per_sm * num_sms();
 }
 
@@ -331,11 +331,11 @@ int default_kv_tile(int d, int nkeys) {
   return 128;
 }
 
-// Validation and dispatch shared by the plain and the ablation entry points.
-template <bool SUMP>
-int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
-                  int N, int d, int causal, int kv_tile, void* o, void* m_out, void* l_out, int* status,
-                  cudaStream_t stream, int l_from_p, float* trace, int two_level) {
+// Host-side checks of an attention call; resolves kv_tile = 0 to the default.  Launches
+// nothing, so an entry point that runs other kernels first (hifa4_attn_fwd quantises V)
+// calls it before them.
+int attn_validate(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
+                  int N, int d, int& kv_tile, const void* o, const int* status) {
   if (!o || !status || !aligned16(o)) return HIFA4_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || N > 63488 || !d_ok(d))
     return HIFA4_ERR_UNSUPPORTED_SHAPE;
@@ -348,6 +348,16 @@ int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qt
     return HIFA4_ERR_INVALID_ARG;
   if ((long long)B * Hq * (N / 128) > 0x7FFFFFFFLL) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  return HIFA4_OK;
+}
+
+// Validation and dispatch shared by the plain and the ablation entry points.
+template <bool SUMP>
+int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
+                  int N, int d, int causal, int kv_tile, void* o, void* m_out, void* l_out, int* status,
+                  cudaStream_t stream, int l_from_p, float* trace, int two_level) {
+  const int rc = attn_validate(q, k, vt, B, Hq, Hkv, N, d, kv_tile, o, status);
+  if (rc != HIFA4_OK) return rc;
 #define HIFA4_LAUNCH(DD, BB) \
   launch_attn<DD, BB, SUMP>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, l_from_p, trace, \
                             nullptr, two_level)
@@ -660,7 +670,7 @@ size_t hifa4_attn_workspace_bytes(int B, int Hkv, int N, int d) {
 int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v, const int64_t v_strides[3],
                    int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* workspace,
                    size_t workspace_bytes, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream) {
-  if (!workspace || !aligned16(workspace)) return HIFA4_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || !strides_ok(v, v_strides)) return HIFA4_ERR_INVALID_ARG;
   if (B <= 0 || Hkv <= 0 || N <= 0 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (workspace_bytes < hifa4_attn_workspace_bytes(B, Hkv, N, d)) return HIFA4_ERR_INVALID_ARG;
   const size_t c = hifa4_qtensor_codes_bytes(B, Hkv, N, d);
@@ -672,7 +682,11 @@ int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v
   vt.N = N;
   vt.d = d;
   vt.transposed = 1;
-  int r = hifa4_quantize_v(v, v_strides, B, Hkv, N, d, &vt, status, stream);
+  // every check of the attention call before the V quantiser launches
+  int tile = kv_tile;
+  int r = attn_validate(q, k, &vt, B, Hq, Hkv, N, d, tile, o, status);
+  if (r != HIFA4_OK) return r;
+  r = hifa4_quantize_v(v, v_strides, B, Hkv, N, d, &vt, status, stream);
   if (r != HIFA4_OK) return r;
   return hifa4_attn_fwd_quantized(q, k, &vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream);
 }

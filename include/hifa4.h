@@ -34,6 +34,9 @@
  *     the FP16 range (|.| > 65504) are outside the supported input range.
  *   - Requires an sm_100 device (B200); anything else returns
  *     HIFA4_ERR_UNSUPPORTED_DEVICE.  There is no CPU fallback.
+ *   - Each kernel's shared-memory attributes and resident-CTA count are set up on its
+ *     first launch and kept for the life of the process (thread-safe), so a process
+ *     drives one GPU, or several identical ones.
  */
 #ifndef HIFA4_H
 #define HIFA4_H

@@ -62,6 +62,33 @@ def test_host_validation_rejects_before_launch(L):
                                       p, None, None, status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
 
 
+def test_attn_fwd_checks_the_attention_before_quantising_v(L):
+    # hifa4_attn_fwd quantises V into its workspace and then runs the attention; a call
+    # the attention would reject must be rejected before the V quantiser is launched (on a
+    # machine without a GPU that launch attempt would report UNSUPPORTED_DEVICE instead)
+    buf = np.zeros(1 << 16, np.uint8)
+    p = ctypes.c_void_p(((buf.ctypes.data + 15) // 16) * 16)
+    status = ctypes.c_void_p(p.value + 32768)
+    st = (ctypes.c_int64 * 3)(0, 128 * 128, 128)
+    ws = L.hifa4_attn_workspace_bytes(1, 2, 128, 128)
+    q = hifa4._QT(p, p, 1, 3, 128, 128, 0)
+    k = hifa4._QT(p, p, 1, 2, 128, 128, 0)
+    # Hq = 3 is not a multiple of Hkv = 2
+    assert L.hifa4_attn_fwd(ctypes.byref(q), ctypes.byref(k), p, st, 1, 3, 2, 128, 128, 1, 0, p, ws, p, None, None,
+                            status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    # a kv tile the head dim does not support
+    q = hifa4._QT(p, p, 1, 2, 128, 128, 0)
+    assert L.hifa4_attn_fwd(ctypes.byref(q), ctypes.byref(k), p, st, 1, 2, 2, 128, 128, 1, 32, p, ws, p, None, None,
+                            status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    # a query tensor whose shape does not match the call
+    qbad = hifa4._QT(p, p, 1, 2, 256, 128, 0)
+    assert L.hifa4_attn_fwd(ctypes.byref(qbad), ctypes.byref(k), p, st, 1, 2, 2, 128, 128, 1, 0, p, ws, p, None,
+                            None, status, None) == hifa4.ERR_INVALID_ARG
+    # a workspace too small for V^T
+    assert L.hifa4_attn_fwd(ctypes.byref(q), ctypes.byref(k), p, st, 1, 2, 2, 128, 128, 1, 0, p, ws - 16, p, None,
+                            None, status, None) == hifa4.ERR_INVALID_ARG
+
+
 def test_layout_permutations_roundtrip():
     rng = np.random.default_rng(0)
     B, H, N, d = 2, 3, 256, 128
