@@ -93,6 +93,40 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _need(t, dtype, what, shape=None, contiguous=False):
+    """Raise unless `t` is a CUDA tensor of `dtype` (and `shape`, and contiguous when
+    asked): the library takes raw device pointers and cannot tell a host buffer or a
+    tensor of another type from the one it expects."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype != dtype:
+        raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{what}: must be on a CUDA device, is on {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+    return t
+
+
+def _need_opt(t, dtype, what, shape=None):
+    return None if t is None else _need(t, dtype, what, shape, contiguous=True)
+
+
+def _need_qt(t, what):
+    if not isinstance(t, QTensor):
+        raise TypeError(f"{what}: expected a QTensor, got {type(t).__name__}")
+    _need(t.codes, torch.uint8, what + ".codes", contiguous=True)
+    _need(t.scales, torch.uint8, what + ".scales", contiguous=True)
+    return t
+
+
+def _smooth(s, sinv, Hkv, d):
+    _need_opt(s, torch.float32, "s", (Hkv, d))
+    _need_opt(sinv, torch.float32, "sinv", (Hkv, d))
+
+
 def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
@@ -124,7 +158,13 @@ def new_status(device=None):
     return torch.zeros(1, dtype=torch.int32, device=device)
 
 
+def _status(status, device):
+    """The caller's device status word (int32, checked) or a new zeroed one."""
+    return new_status(device) if status is None else _need(status, torch.int32, "status")
+
+
 def hifa4_read_status(status, clear=True):
+    _need(status, torch.int32, "status")
     return lib().hifa4_read_status(_ptr(status), int(clear), _stream())
 
 
@@ -138,6 +178,8 @@ def hifa4_debug_set_injection(mode: int):
 
 def hifa4_calibrate_smooth(q_cal, k_cal, alpha: float):
     """Smooth-QK scales (s, s_inv), fp32 [Hkv, d] on q_cal's device.  Synchronises."""
+    _need(q_cal, torch.bfloat16, "q_cal")
+    _need(k_cal, torch.bfloat16, "k_cal")
     B, Hq, N, d = q_cal.shape
     Hkv = k_cal.shape[1]
     dev = q_cal.device
@@ -151,11 +193,14 @@ def hifa4_calibrate_smooth(q_cal, k_cal, alpha: float):
 
 def hifa4_quantize_qk(q, k, s=None, sinv=None, status=None, out=None):
     """Smooth-QK + 4-bit quantisation of bf16 Q [B,Hq,N,d] and K [B,Hkv,N,d] -> (QTensor, QTensor)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
+    _smooth(s, sinv, Hkv, d)
     if out is None:
         out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device))
-    st = status if status is not None else new_status(q.device)
+    st = _status(status, q.device)
     _check(lib().hifa4_quantize_qk(_ptr(q), _ptr(k), _strides(q), _strides(k), B, Hq, Hkv, N, d, _ptr(s), _ptr(sinv),
                                    out[0].c(), out[1].c(), _ptr(st), _stream()), "hifa4_quantize_qk")
     return out
@@ -174,11 +219,16 @@ def hifa4_rope_table(theta: float, N: int, d: int, pos0: int = 0):
 def hifa4_quantize_qk_rope(q, k, rope_cos, rope_sin, s=None, sinv=None, status=None, out=None):
     """Fused RoPE + Smooth-QK + 4-bit quantisation of PRE-RoPE bf16 Q [B,Hq,N,d] and K
     [B,Hkv,N,d]; rope_cos, rope_sin: device fp32 [N, d/2] -> (QTensor, QTensor)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
+    _need(rope_cos, torch.float32, "rope_cos", (N, d // 2), contiguous=True)
+    _need(rope_sin, torch.float32, "rope_sin", (N, d // 2), contiguous=True)
+    _smooth(s, sinv, Hkv, d)
     if out is None:
         out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device))
-    st = status if status is not None else new_status(q.device)
+    st = _status(status, q.device)
     _check(lib().hifa4_quantize_qk_rope(_ptr(q), _ptr(k), _strides(q), _strides(k), B, Hq, Hkv, N, d, _ptr(rope_cos),
                                         _ptr(rope_sin), _ptr(s), _ptr(sinv), out[0].c(), out[1].c(), _ptr(st),
                                         _stream()), "hifa4_quantize_qk_rope")
@@ -187,11 +237,15 @@ def hifa4_quantize_qk_rope(q, k, rope_cos, rope_sin, s=None, sinv=None, status=N
 
 def hifa4_quantize_qkv(q, k, v, s=None, sinv=None, status=None, out=None):
     """Smooth-QK + 4-bit Q, K and V^T in one launch -> (QTensor, QTensor, QTensor)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    _need(v, torch.bfloat16, "v")
     B, Hq, N, d = q.shape
     Hkv = k.shape[1]
+    _smooth(s, sinv, Hkv, d)
     if out is None:
         out = (QTensor(B, Hq, N, d, 0, q.device), QTensor(B, Hkv, N, d, 0, q.device), QTensor(B, Hkv, N, d, 1, q.device))
-    st = status if status is not None else new_status(q.device)
+    st = _status(status, q.device)
     _check(lib().hifa4_quantize_qkv(_ptr(q), _ptr(k), _ptr(v), _strides(q), _strides(k), _strides(v), B, Hq, Hkv, N, d,
                                     _ptr(s), _ptr(sinv), out[0].c(), out[1].c(), out[2].c(), _ptr(st), _stream()),
            "hifa4_quantize_qkv")
@@ -200,28 +254,36 @@ def hifa4_quantize_qkv(q, k, v, s=None, sinv=None, status=None, out=None):
 
 def hifa4_quantize_v(v, status=None, out=None):
     """4-bit quantisation of V^T (blocks of 16 tokens) of bf16 V [B,Hkv,N,d] -> QTensor."""
+    _need(v, torch.bfloat16, "v")
     B, Hkv, N, d = v.shape
     out = out if out is not None else QTensor(B, Hkv, N, d, 1, v.device)
-    st = status if status is not None else new_status(v.device)
+    st = _status(status, v.device)
     _check(lib().hifa4_quantize_v(_ptr(v), _strides(v), B, Hkv, N, d, out.c(), _ptr(st), _stream()), "hifa4_quantize_v")
     return out
 
 
-def _outputs(qq, dev, o, m, l):
-    B, Hq, N, d = qq.B, qq.H, qq.N, qq.d
+def _outputs(B, Hq, N, d, dev, o, m, l):
+    """Output tensors o bf16 [B, Hq, N, d], m and l fp16 [B, Hq, N]: the given ones after
+    checking them, else new ones."""
     if o is None:
         o = torch.empty(B, Hq, N, d, dtype=torch.bfloat16, device=dev)
     if m is None:
         m = torch.empty(B, Hq, N, dtype=torch.float16, device=dev)
     if l is None:
         l = torch.empty(B, Hq, N, dtype=torch.float16, device=dev)
+    _need(o, torch.bfloat16, "o", (B, Hq, N, d), contiguous=True)
+    _need(m, torch.float16, "m", (B, Hq, N), contiguous=True)
+    _need(l, torch.float16, "l", (B, Hq, N), contiguous=True)
     return o, m, l
 
 
 def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=None, m=None, l=None):
+    """The fused 4-bit attention of already quantised Q, K and V^T -> (O bf16, m fp16, l fp16)."""
+    for t, w in ((qq, "q"), (kq, "k"), (vt, "vt")):
+        _need_qt(t, w)
     dev = qq.codes.device
-    o, m, l = _outputs(qq, dev, o, m, l)
-    st = status if status is not None else new_status(dev)
+    o, m, l = _outputs(qq.B, qq.H, qq.N, qq.d, dev, o, m, l)
+    st = _status(status, dev)
     _check(lib().hifa4_attn_fwd_quantized(qq.c(), kq.c(), vt.c(), qq.B, qq.H, kq.H, qq.N, qq.d, int(causal),
                                           int(kv_tile), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
            "hifa4_attn_fwd_quantized")
@@ -234,12 +296,16 @@ def hifa4_attn_fwd_ablation(q: QTensor, k: QTensor, vt: QTensor, causal: bool, k
     P_hat), 1 = the inconsistent formulation (sum of unquantised P); two_level selects the
     two-level P scale (a per-row, per-tile power of two under the block scales of P).
     trace: optional fp32 [B, Hq, N, N/kv_tile, 2] receiving (sum P_hat, sum P) per (row, tile)."""
-    import torch
+    for t, w in ((q, "q"), (k, "k"), (vt, "vt")):
+        _need_qt(t, w)
     dev = q.codes.device
-    o = o if o is not None else torch.empty(q.B, q.H, q.N, q.d, dtype=torch.bfloat16, device=dev)
-    m = m if m is not None else torch.empty(q.B, q.H, q.N, dtype=torch.float16, device=dev)
-    l = l if l is not None else torch.empty(q.B, q.H, q.N, dtype=torch.float16, device=dev)
-    st = status if status is not None else new_status(dev)
+    o, m, l = _outputs(q.B, q.H, q.N, q.d, dev, o, m, l)
+    if trace is not None:
+        nt = q.N // (kv_tile if kv_tile else (256 if q.d == 128 and q.N % 256 == 0 else (64 if q.d == 256 else 128)))
+        _need(trace, torch.float32, "trace", contiguous=True)
+        if trace.numel() != q.B * q.H * q.N * nt * 2:
+            raise ValueError(f"trace: expected {q.B * q.H * q.N * nt * 2} elements, got {trace.numel()}")
+    st = _status(status, dev)
     _check(lib().hifa4_attn_fwd_ablation(q.c(), k.c(), vt.c(), q.B, q.H, k.H, q.N, q.d, int(causal), int(kv_tile),
                                          int(normaliser), int(bool(two_level)), _ptr(trace), _ptr(o), _ptr(m), _ptr(l),
                                          _ptr(st), _stream()),
@@ -250,9 +316,11 @@ def hifa4_attn_fwd_ablation(q: QTensor, k: QTensor, vt: QTensor, causal: bool, k
 def hifa4_quantize_q_decode(q, Hkv: int, s=None, status=None, out=None):
     """Smooth-QK + 4-bit quantisation of a decode query bf16 [B, Hq, nq, d] into the packed
     [B, Hkv, 128, d] QTensor (row hi * nq + t = token t of query head g * G + hi)."""
+    _need(q, torch.bfloat16, "q")
     B, Hq, nq, d = q.shape
+    _need_opt(s, torch.float32, "s", (Hkv, d))
     out = out if out is not None else QTensor(B, Hkv, 128, d, 0, q.device)
-    st = status if status is not None else new_status(q.device)
+    st = _status(status, q.device)
     _check(lib().hifa4_quantize_q_decode(_ptr(q), _strides(q), B, Hq, Hkv, nq, d, _ptr(s), out.c(), _ptr(st),
                                          _stream()), "hifa4_quantize_q_decode")
     return out
@@ -262,17 +330,17 @@ def hifa4_attn_decode(q: QTensor, k: QTensor, vt: QTensor, Hq: int, nq: int, kv_
                       status=None, workspace=None, o=None, m=None, l=None):
     """Decode / split-KV attention of the packed query q against K, V^T of Nk = k.N keys ->
     (o bf16 [B, Hq, nq, d], m, l fp16 [B, Hq, nq])."""
-    import torch
+    for t, w in ((q, "q"), (k, "k"), (vt, "vt")):
+        _need_qt(t, w)
     dev = q.codes.device
     B, Hkv, Nk, d = k.B, k.H, k.N, k.d
     ns = nsplit if nsplit > 0 else 64
     need = lib().hifa4_decode_workspace_bytes(B, Hkv, ns, d)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    o = o if o is not None else torch.empty(B, Hq, nq, d, dtype=torch.bfloat16, device=dev)
-    m = m if m is not None else torch.empty(B, Hq, nq, dtype=torch.float16, device=dev)
-    l = l if l is not None else torch.empty(B, Hq, nq, dtype=torch.float16, device=dev)
-    st = status if status is not None else new_status(dev)
+    _need(workspace, torch.uint8, "workspace", contiguous=True)
+    o, m, l = _outputs(B, Hq, nq, d, dev, o, m, l)
+    st = _status(status, dev)
     _check(lib().hifa4_attn_decode(q.c(), k.c(), vt.c(), B, Hq, Hkv, nq, Nk, d, int(kv_tile), int(nsplit),
                                    _ptr(workspace), workspace.numel(), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
            "hifa4_attn_decode")
@@ -281,13 +349,17 @@ def hifa4_attn_decode(q: QTensor, k: QTensor, vt: QTensor, Hq: int, nq: int, kv_
 
 def hifa4_attn_fwd(qq, kq, v, causal=True, kv_tile=0, status=None, workspace=None, o=None, m=None, l=None):
     """Quantise V^T into a workspace and run the fused 4-bit attention -> (O bf16, m fp16, l fp16)."""
+    _need_qt(qq, "q")
+    _need_qt(kq, "k")
+    _need(v, torch.bfloat16, "v")
     B, Hkv, N, d = v.shape
     dev = v.device
-    o, m, l = _outputs(qq, dev, o, m, l)
+    o, m, l = _outputs(qq.B, qq.H, qq.N, qq.d, dev, o, m, l)
     need = lib().hifa4_attn_workspace_bytes(B, Hkv, N, d)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    st = status if status is not None else new_status(dev)
+    _need(workspace, torch.uint8, "workspace", contiguous=True)
+    st = _status(status, dev)
     _check(lib().hifa4_attn_fwd(qq.c(), kq.c(), _ptr(v), _strides(v), qq.B, qq.H, Hkv, N, d, int(causal), int(kv_tile),
                                 _ptr(workspace), workspace.numel(), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
            "hifa4_attn_fwd")
@@ -299,23 +371,28 @@ def hifa4_attn_workspace_bytes(B, Hkv, N, d):
 
 
 def hifa4_probe_qk_tile(q_codes, q_scales, k_codes, k_scales, d, kv_tile, status=None):
+    for t, w in ((q_codes, "q_codes"), (q_scales, "q_scales"), (k_codes, "k_codes"), (k_scales, "k_scales")):
+        _need(t, torch.uint8, w, contiguous=True)
     S = torch.empty(128, kv_tile, dtype=torch.float32, device=q_codes.device)
-    st = status if status is not None else new_status(q_codes.device)
+    st = _status(status, q_codes.device)
     _check(lib().hifa4_probe_qk_tile(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), d, kv_tile, _ptr(S),
                                      _ptr(st), _stream()), "hifa4_probe_qk_tile")
     return S
 
 
 def hifa4_probe_pv_tile(p_codes, p_scales, vt_codes, vt_scales, d, kv_tile, status=None):
+    for t, w in ((p_codes, "p_codes"), (p_scales, "p_scales"), (vt_codes, "vt_codes"), (vt_scales, "vt_scales")):
+        _need(t, torch.uint8, w, contiguous=True)
     O = torch.empty(128, d, dtype=torch.float32, device=p_codes.device)
     R = torch.empty(128, dtype=torch.float32, device=p_codes.device)
-    st = status if status is not None else new_status(p_codes.device)
+    st = _status(status, p_codes.device)
     _check(lib().hifa4_probe_pv_tile(_ptr(p_codes), _ptr(p_scales), _ptr(vt_codes), _ptr(vt_scales), d, kv_tile, _ptr(O),
                                      _ptr(R), _ptr(st), _stream()), "hifa4_probe_pv_tile")
     return O, R
 
 
 def hifa4_probe_codec(x):
+    _need(x, torch.float32, "x", contiguous=True)
     n = x.numel()
     e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
     e4 = torch.empty(n, dtype=torch.uint8, device=x.device)

@@ -62,6 +62,33 @@ def test_host_validation_rejects_before_launch(L):
                                       p, None, None, status, None) == hifa4.ERR_UNSUPPORTED_SHAPE
 
 
+def test_fused_rope_quantiser_rejects_null_tables(L):
+    buf = np.zeros(4096, np.uint8)
+    p = ctypes.c_void_p(((buf.ctypes.data + 15) // 16) * 16)
+    status = ctypes.c_void_p(p.value + 2048)
+    st = (ctypes.c_int64 * 3)(0, 0, 128)
+    qt = hifa4._QT(p, p, 1, 1, 128, 128, 0)
+    assert L.hifa4_quantize_qk_rope(p, p, st, st, 1, 1, 1, 128, 128, None, None, None, None, ctypes.byref(qt),
+                                    ctypes.byref(qt), status, None) == hifa4.ERR_INVALID_ARG
+    assert L.hifa4_quantize_qk_rope(p, p, st, st, 1, 1, 1, 128, 128, p, ctypes.c_void_p(p.value + 4), None, None,
+                                    ctypes.byref(qt), ctypes.byref(qt), status, None) == hifa4.ERR_INVALID_ARG
+
+
+def test_binding_checks_tensors_before_the_call():
+    # the binding hands raw device pointers to the library; host tensors and tensors of
+    # another type are refused before any call
+    import torch
+    x = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        hifa4.hifa4_quantize_v(x)
+    with pytest.raises(TypeError, match="bfloat16"):
+        hifa4.hifa4_quantize_v(x.float())
+    with pytest.raises(TypeError, match="QTensor"):
+        hifa4.hifa4_attn_fwd_quantized(x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        hifa4.hifa4_read_status(torch.zeros(1, dtype=torch.int32))
+
+
 def test_attn_fwd_checks_the_attention_before_quantising_v(L):
     # hifa4_attn_fwd quantises V into its workspace and then runs the attention; a call
     # the attention would reject must be rejected before the V quantiser is launched (on a

@@ -95,9 +95,16 @@ def test_attention_on_fused_quantised_inputs():
 
 
 def test_fused_rope_rejects_bad_tables():
+    # the binding checks the tables' type, shape and placement before the call (the C
+    # ABI's own check of null tables is a CPU test)
     q = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(hifa4.Hifa4Error):
+    with pytest.raises(TypeError):
         hifa4.hifa4_quantize_qk_rope(q, q, None, None)
+    cos, sin = hifa4.hifa4_rope_table(1e4, 128, 128)
+    with pytest.raises(ValueError):     # host tables
+        hifa4.hifa4_quantize_qk_rope(q, q, torch.from_numpy(cos), torch.from_numpy(sin))
+    with pytest.raises(ValueError):     # tables of another length
+        hifa4.hifa4_quantize_qk_rope(q, q, gc.to_dev(cos[:64]), gc.to_dev(sin[:64]))
 
 
 def test_exact_cancellations_give_positive_zero():
