@@ -30,7 +30,7 @@ FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput rat
 # DRAM bytes (read + write) of one k_attn_fwd<128, 256> launch on qwen3-8b-4k, from an ncu
 # capture of this kernel version (dram__bytes_read.sum + dram__bytes_write.sum; summary and
 # command in profiles/attn_fwd_qwen3-8b-4k.md).  Set to None when the kernel changes.
-ATTN_TRAFFIC_BYTES = 14.216e6 + 0.072e6
+ATTN_TRAFFIC_BYTES = 14.217472e6 + 0.1216e6
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 
