@@ -3,14 +3,15 @@
 One step = the whole hot path over one batch of the Qwen3-8B-shaped 4k causal workload
 (B=1, Hq=32, Hkv=8, N=4096, d=128): Smooth-QK + 4-bit quantisation of Q and K and 4-bit
 quantisation of V^T (one launch, hifa4_quantize_qkv), then the fused 4-bit attention
-kernel (hifa4_attn_fwd_quantized), both through the C ABI (libhifa4.so).  Metric: TFLOPS = 4*B*Hq*N^2*d / 2 (causal) per step / step time.
+kernel (hifa4_attn_fwd_quantized), both through the C ABI (libhifa4.so).
+Metric: TFLOPS = 4*B*Hq*N^2*d / 2 (causal) per step / step time.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 
 Under torchrun (N > 1) every rank runs the same per-GPU workload (weak scaling, no
 collective on the data path); value = flops of all ranks / max-over-ranks time.
---impl reference times the CPU oracle (the reference arm of this build) on a bounded
-sample of the same workload.
+--impl reference times the CPU oracle (the method's plain CPU implementation, the only
+reference there is) on a bounded sample of the same workload.
 """
 import argparse
 import json
