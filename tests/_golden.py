@@ -1,0 +1,44 @@
+"""Reader of the hand-derived worked examples in tests/golden/worked_examples.txt and the
+input recipe of its attention cases (shared by the oracle and GPU tests)."""
+import os
+
+import numpy as np
+
+from bit_flashattention_b200 import gen
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "worked_examples.txt")
+
+
+def load():
+    """{section: {key: [tokens]}} of the fixture ('#' comments dropped)."""
+    sections, cur = {}, None
+    for raw in open(GOLDEN):
+        line = raw.split("#", 1)[0].strip()
+        if not line:
+            continue
+        if line.startswith("[") and line.endswith("]"):
+            cur = sections.setdefault(line[1:-1], {})
+            continue
+        key, val = line.split(":", 1)
+        cur[key.strip()] = val.split()
+    return sections
+
+
+def num(s):
+    return int(s, 16) if s.startswith("0x") else float(s)
+
+
+# the 16 E2M1 multiples every 16-token block of a V channel holds (a rotation of them)
+L = np.array([6, -6, 4, -4, 3, -3, 2, -2, 1.5, -1.5, 1, -1, 0.5, -0.5, 0, 6], np.float64)
+
+
+def attn_inputs(N=256, d=64):
+    """The fixture's attention inputs as bf16 bits [1, 1, N, d]: Q = 0, K any values,
+    V[n, c] = 2^-(c % 4) / 4 * L[(n + c) % 16]; also V as float64 [N, d]."""
+    n = np.arange(N)[:, None]
+    c = np.arange(d)[None, :]
+    v = np.exp2(-(c % 4)) / 4 * L[(n + c) % 16]
+    k = ((7 * n + 3 * c) % 13 - 6) * 0.5              # any values: Q_hat = 0 ignores them
+    q = np.zeros((N, d))
+    bits = lambda a: gen.f32_to_bf16_bits(a.astype(np.float32))[None, None]
+    return bits(q), bits(k), bits(v), v

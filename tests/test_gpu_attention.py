@@ -159,3 +159,32 @@ def test_default_kv_tile_when_n_is_not_a_multiple_of_256():
     rows = np.arange(w.B * w.Hq * w.N, dtype=np.int64)
     ref = oracle.attn_fwd(qz, True, 128, rows)
     gc.assert_parity(gc.compare_outputs(w, rows, o0, m0, l0, ref))
+
+
+@pytest.mark.parametrize("kv_tile", [64, 128])
+def test_worked_examples_from_the_golden_fixture(kv_tile):
+    # the hand-derived attention cases of tests/golden/worked_examples.txt on the GPU:
+    # Q = 0 over a V that quantises exactly gives m = 0, l = 264 and O = 0.09375 * 2^-(c%4)
+    # on every row; the first causal row gives l = 1.03125 and O = V[0]
+    from tests import _golden
+    G = _golden.load()
+    q, k, v, vf = _golden.attn_inputs()
+    qq, kq, vq, vt = gc.gpu_quantize(configs.scaled(configs.get("tiny"), N=256, d=64, bc=kv_tile), q, k, v, None,
+                                     None)
+    bits = lambda t: t.reshape(t.shape[0] * t.shape[1] * t.shape[2], -1).view(torch.int16).cpu().numpy().view(np.uint16)
+    st = hifa4.new_status("cuda")
+    o, m, l = hifa4.hifa4_attn_fwd(qq, kq, vt, causal=False, kv_tile=kv_tile, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    sec = G["attn_q_zero"]
+    assert np.all(bits(m[..., None]) == _golden.num(sec["m_fp16"][0]))
+    assert np.all(bits(l[..., None]) == _golden.num(sec["l_fp16"][0]))
+    want = np.array([_golden.num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(64) % 4]
+    assert np.all(bits(o) == want[None, :])
+    o, m, l = hifa4.hifa4_attn_fwd(qq, kq, vt, causal=True, kv_tile=kv_tile, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    sec = G["attn_causal_row0"]
+    assert bits(m[..., None])[0, 0] == _golden.num(sec["m_fp16"][0])
+    assert bits(l[..., None])[0, 0] == _golden.num(sec["l_fp16"][0])
+    o0 = o[0, 0, 0].float().cpu().numpy()
+    assert o0[:16].tolist() == [float(x) for x in sec["o_first_16"]]
+    assert np.array_equal(o0, vf[0].astype(np.float32))
