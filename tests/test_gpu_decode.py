@@ -139,3 +139,25 @@ def test_decode_rejects_bad_shapes():
     q = torch.zeros(1, 8, 33, 128, dtype=torch.bfloat16, device="cuda")     # G * nq = 132 > 128
     with pytest.raises(hifa4.Hifa4Error):
         hifa4.hifa4_quantize_q_decode(q, 2, status=st)
+
+
+@pytest.mark.parametrize("d,kv_tile,nsplit", [(128, 0, 1), (128, 0, 2), (128, 256, 1), (64, 64, 3)])
+def test_decode_worked_example_from_the_golden_fixture(d, kv_tile, nsplit):
+    # the hand-derived decode case of tests/golden/worked_examples.txt: Q = 0 against the
+    # fixture's V over 256 keys gives m = 0, l = 264 and O = 0.09375 * 2^-(c % 4) at any
+    # split count (kv_tile 0 at d = 128: the kernel with the keys on the MMA's M dimension)
+    from tests import _golden
+    sec = _golden.load()["decode_q_zero"]
+    _, k, v, _ = _golden.attn_inputs(256, d)
+    st = hifa4.new_status("cuda")
+    q = torch.zeros(1, 1, 1, d, dtype=torch.bfloat16, device="cuda")
+    qp = hifa4.hifa4_quantize_q_decode(q, 1, status=st)
+    kq, _ = hifa4.hifa4_quantize_qk(gc.bf16_dev(k), gc.bf16_dev(k), status=st)
+    vq = hifa4.hifa4_quantize_v(gc.bf16_dev(v), status=st)
+    o, m, l = hifa4.hifa4_attn_decode(qp, kq, vq, 1, 1, kv_tile=kv_tile, nsplit=nsplit, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    u16 = lambda t: t.reshape(-1).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert u16(m)[0] == _golden.num(sec["m_fp16"][0])
+    assert u16(l)[0] == _golden.num(sec["l_fp16"][0])
+    want = np.array([_golden.num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(d) % 4]
+    assert np.array_equal(u16(o), want)

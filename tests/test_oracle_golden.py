@@ -15,7 +15,7 @@ G = load()
 
 def test_fixture_has_every_section():
     assert set(G) == {"e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode", "block_exact", "block_flushed",
-                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0"}
+                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0", "decode_q_zero"}
 
 
 def test_e2m1_decode(orc):
@@ -100,3 +100,18 @@ def test_first_causal_row(orc):
     assert np.array_equal(got, vf[0].astype(np.float32))
     t = orc.attn_trace(orc.quantize_all(q, k, v), True, 64, 0)
     assert t["phat"].shape == (1, 64) and t["phat"][0, 0] == 1.03125 and np.all(t["phat"][0, 1:] == 0)
+
+
+@pytest.mark.parametrize("d,bc,nsplit", [(64, 64, 1), (64, 64, 3), (128, 128, 2), (128, 256, 1), (128, 16, 16)])
+def test_decode_with_zero_query(orc, d, bc, nsplit):
+    sec = G["decode_q_zero"]
+    _, k, v, _ = _attn_inputs(256, d)
+    q = np.zeros((1, 1, 1, d), np.uint16)
+    qc, qs = orc.quantize_rows(orc.pack_decode_q(q, 1), 1)
+    kc, ks = orc.quantize_rows(k, 1)
+    vc, vs = orc.quantize_vt(v)
+    ref = orc.attn_decode(qc, qs, kc, ks, vc, vs, G=1, nq=1, bc=bc, nsplit=nsplit)
+    assert ref["m"].astype(np.float16).view(np.uint16)[0, 0, 0] == _num(sec["m_fp16"][0])
+    assert ref["l"].astype(np.float16).view(np.uint16)[0, 0, 0] == _num(sec["l_fp16"][0])
+    want = np.array([_num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(d) % 4]
+    assert np.array_equal(ref["o_bf16"][0, 0, 0], want)
