@@ -42,3 +42,17 @@ def attn_inputs(N=256, d=64):
     q = np.zeros((N, d))
     bits = lambda a: gen.f32_to_bf16_bits(a.astype(np.float32))[None, None]
     return bits(q), bits(k), bits(v), v
+
+
+def select_inputs(N=256, d=64):
+    """The attn_select case: every query row (6, 0, ..., 0); key n with n % 4 == 0 zero in
+    channels 0..15, the others -6 in channel 0 and zero in 1..15; channels 16.. of K any
+    values; V as in attn_inputs.  bf16 bits [1, 1, N, d]."""
+    _, k, v, vf = attn_inputs(N, d)
+    kf = gen.bf16_bits_to_f32(k[0, 0]).copy()
+    kf[:, :16] = 0.0
+    kf[np.arange(N) % 4 != 0, 0] = -6.0
+    q = np.zeros((N, d), np.float32)
+    q[:, 0] = 6.0
+    bits = lambda a: gen.f32_to_bf16_bits(a.astype(np.float32))[None, None]
+    return bits(q), bits(kf), v, vf

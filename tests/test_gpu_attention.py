@@ -188,3 +188,21 @@ def test_worked_examples_from_the_golden_fixture(kv_tile):
     o0 = o[0, 0, 0].float().cpu().numpy()
     assert o0[:16].tolist() == [float(x) for x in sec["o_first_16"]]
     assert np.array_equal(o0, vf[0].astype(np.float32))
+
+
+@pytest.mark.parametrize("kv_tile", [64, 128])
+def test_selected_keys_worked_example_from_the_golden_fixture(kv_tile):
+    # the fixture's attn_select case: nonzero scores (S = 0 or -36) through both 4-bit
+    # GEMMs; P_hat = 1.03125 on every fourth key and 0 elsewhere, l = 66, O exact in bf16
+    from tests import _golden
+    sec = _golden.load()["attn_select"]
+    q, k, v, _ = _golden.select_inputs()
+    qq, kq, vq, vt = gc.gpu_quantize(None, q, k, v, None, None)
+    st = hifa4.new_status("cuda")
+    o, m, l = hifa4.hifa4_attn_fwd(qq, kq, vt, causal=False, kv_tile=kv_tile, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    u16 = lambda t: t.reshape(t.shape[2], -1).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.all(u16(m[..., None]) == _golden.num(sec["m_fp16"][0]))
+    assert np.all(u16(l[..., None]) == _golden.num(sec["l_fp16"][0]))
+    want = np.array([_golden.num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(64) % 4]
+    assert np.all(u16(o) == want[None, :])

@@ -15,7 +15,7 @@ G = load()
 
 def test_fixture_has_every_section():
     assert set(G) == {"e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode", "block_exact", "block_flushed",
-                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0", "decode_q_zero"}
+                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0", "decode_q_zero", "attn_select"}
 
 
 def test_e2m1_decode(orc):
@@ -115,3 +115,22 @@ def test_decode_with_zero_query(orc, d, bc, nsplit):
     assert ref["l"].astype(np.float16).view(np.uint16)[0, 0, 0] == _num(sec["l_fp16"][0])
     want = np.array([_num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(d) % 4]
     assert np.array_equal(ref["o_bf16"][0, 0, 0], want)
+
+
+@pytest.mark.parametrize("bc", [16, 64, 256])
+def test_attention_over_selected_keys(orc, bc):
+    from tests import _golden
+    sec = G["attn_select"]
+    q, k, v, _ = _golden.select_inputs()
+    qz = orc.quantize_all(q, k, v)
+    assert qz.qs[0, 0, 0, 0] == 0x38 and qz.qc[0, 0, 0, 0] == 7
+    assert np.all(qz.ks[0, 0, 1::4, 0] == 0x38) and np.all(qz.ks[0, 0, 0::4, 0] == 0)
+    ref = orc.attn_fwd(qz, False, bc)
+    assert np.all(ref["m16"] == _num(sec["m_fp16"][0]))
+    assert np.all(ref["l16"] == _num(sec["l_fp16"][0]))
+    want = np.array([_num(b) for b in sec["o_bf16_by_c_mod_4"]], np.uint16)[np.arange(64) % 4]
+    assert np.all(ref["o_bf16"] == want[None, :]), ref["o_bf16"][0][:4]
+    t = orc.attn_trace(qz, False, bc, 5)
+    sel = (np.arange(256) % 4 == 0).reshape(-1, bc)
+    assert np.all(t["phat"][sel] == 1.03125) and np.all(t["phat"][~sel] == 0)
+    assert np.all(np.abs(t["p"][~sel] - 2.0 ** (-36 * np.float32(np.log2(np.e) / 8))) < 1e-3)
