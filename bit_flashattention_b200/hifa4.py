@@ -99,11 +99,11 @@ def _need(t, dtype, what, shape=None, contiguous=False):
     tensor of another type from the one it expects."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{what}: expected a torch.Tensor, got {type(t).__name__}")
-    if t.dtype != dtype:
+    if t.dtype is not dtype:
         raise TypeError(f"{what}: expected {dtype}, got {t.dtype}")
-    if t.device.type != "cuda":
+    if not t.is_cuda:
         raise ValueError(f"{what}: must be on a CUDA device, is on {t.device}")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError(f"{what}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
     if contiguous and not t.is_contiguous():
         raise ValueError(f"{what}: must be contiguous")
@@ -115,10 +115,9 @@ def _need_opt(t, dtype, what, shape=None):
 
 
 def _need_qt(t, what):
+    # a QTensor's buffers are checked when it is built
     if not isinstance(t, QTensor):
         raise TypeError(f"{what}: expected a QTensor, got {type(t).__name__}")
-    _need(t.codes, torch.uint8, what + ".codes", contiguous=True)
-    _need(t.scales, torch.uint8, what + ".scales", contiguous=True)
     return t
 
 
@@ -148,6 +147,10 @@ class QTensor:
         ns = L.hifa4_qtensor_scales_bytes(B, H, N, d, self.transposed)
         self.codes = codes if codes is not None else torch.empty(nc, dtype=torch.uint8, device=device)
         self.scales = scales if scales is not None else torch.empty(ns, dtype=torch.uint8, device=device)
+        for t, w, n in ((self.codes, "codes", nc), (self.scales, "scales", ns)):
+            _need(t, torch.uint8, "QTensor." + w, contiguous=True)
+            if t.numel() < n:
+                raise ValueError(f"QTensor.{w}: {t.numel()} bytes, the layout needs {n}")
 
     def c(self):
         return ctypes.byref(_QT(self.codes.data_ptr(), self.scales.data_ptr(), self.B, self.H, self.N, self.d,

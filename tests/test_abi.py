@@ -87,6 +87,11 @@ def test_binding_checks_tensors_before_the_call():
         hifa4.hifa4_attn_fwd_quantized(x, x, x)
     with pytest.raises(ValueError, match="CUDA"):
         hifa4.hifa4_read_status(torch.zeros(1, dtype=torch.int32))
+    # a QTensor checks its buffers once, when it is built
+    with pytest.raises(ValueError, match="CUDA"):
+        hifa4.QTensor(1, 1, 128, 128, 0)
+    with pytest.raises(TypeError, match="uint8"):
+        hifa4.QTensor(1, 1, 128, 128, 0, codes=torch.zeros(8192, dtype=torch.int8), scales=None)
 
 
 def test_attn_fwd_checks_the_attention_before_quantising_v(L):
