@@ -56,3 +56,16 @@ def select_inputs(N=256, d=64):
     q[:, 0] = 6.0
     bits = lambda a: gen.f32_to_bf16_bits(a.astype(np.float32))[None, None]
     return bits(q), bits(kf), v, vf
+
+
+def tie_inputs(N=256, d=64):
+    """The attn_bf16_tie case: Q = 0, K as in attn_inputs, every V channel 1 except a 1.5
+    at the start of each 16-token block, then a 1.5 (block 0) or a 0.5 (the others).
+    bf16 bits [1, 1, N, d]."""
+    q, k, _, _ = attn_inputs(N, d)
+    col = np.ones(N)
+    col[0::16] = 1.5
+    col[1::16] = 0.5
+    col[1] = 1.5
+    v = np.repeat(col[:, None], d, axis=1)
+    return q, k, gen.f32_to_bf16_bits(v.astype(np.float32))[None, None]

@@ -147,3 +147,24 @@ def test_mirror_close_to_exact_attention(orc):
     direct = orc.attn_fwd(qz0, True, 128, rows, l_from_p=True, want_f64=True)["o_f64"].reshape(w.Hq, w.N, w.d)
     print(f"\nrelative error vs fp64 attention: HiFA4 {rel(mir, ref):.4f} (operand quantisation alone "
           f"{rel(deq, ref):.4f}), direct FP4 {rel(direct, ref):.4f}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_running_max_is_the_fp16_rounding_of_the_scaled_row_max(orc, causal):
+    # the online-softmax state is FP16: the final m of a row is the FP16 rounding (nearest
+    # even) of the largest RN(S * c) over its visible keys, whatever the tile order, since
+    # that rounding is monotone; m and l are FP16 values
+    w = _small(B=1, Hq=2, Hkv=1, N=256, d=128)
+    qz, _ = _quantized(w)
+    ref = orc.attn_fwd(qz, causal, 64)
+    c = np.float32(np.log2(np.e) / np.sqrt(w.d))
+    for h in range(w.Hq):
+        S = orc.qk_scores(qz.qc[0, h], qz.qs[0, h], qz.kc[0, 0], qz.ks[0, 0])
+        t = (S.astype(np.float32) * c).astype(np.float32)
+        if causal:
+            t = np.where(np.tril(np.ones_like(t, dtype=bool)), t, -np.inf)
+        want = t.max(axis=1).astype(np.float16)
+        got = ref["m"][h * w.N:(h + 1) * w.N]
+        assert np.array_equal(got.astype(np.float16), want)
+        assert np.array_equal(got, want.astype(np.float32))
+    assert np.array_equal(ref["l"], ref["l"].astype(np.float16).astype(np.float32))

@@ -15,7 +15,8 @@ G = load()
 
 def test_fixture_has_every_section():
     assert set(G) == {"e2m1_decode", "e2m1_encode", "e4m3_decode", "e4m3_encode", "block_exact", "block_flushed",
-                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0", "decode_q_zero", "attn_select"}
+                      "block_clipped", "calibration", "attn_q_zero", "attn_causal_row0", "decode_q_zero", "attn_select",
+                      "attn_bf16_tie"}
 
 
 def test_e2m1_decode(orc):
@@ -134,3 +135,16 @@ def test_attention_over_selected_keys(orc, bc):
     sel = (np.arange(256) % 4 == 0).reshape(-1, bc)
     assert np.all(t["phat"][sel] == 1.03125) and np.all(t["phat"][~sel] == 0)
     assert np.all(np.abs(t["p"][~sel] - 2.0 ** (-36 * np.float32(np.log2(np.e) / 8))) < 1e-3)
+
+
+@pytest.mark.parametrize("bc", [64, 256])
+def test_output_rounds_a_tie_to_even(orc, bc):
+    from tests import _golden
+    sec = G["attn_bf16_tie"]
+    q, k, v = _golden.tie_inputs()
+    qz = orc.quantize_all(q, k, v)
+    assert np.all(qz.vs == 0x28)
+    ref = orc.attn_fwd(qz, False, bc, want_f64=True)
+    assert np.all(ref["m16"] == _num(sec["m_fp16"][0])) and np.all(ref["l16"] == _num(sec["l_fp16"][0]))
+    assert np.all(ref["o_f64"] == 1.0 + 2.0 ** -8)          # O / l before the bf16 rounding
+    assert np.all(ref["o_bf16"] == _num(sec["o_bf16"][0]))
