@@ -474,10 +474,12 @@ def run_reference(args):
     w = configs.get(WORKLOAD)
     data = _oracle_setup(w)
     nqt = w.N // 128
-    for i in range(min(args.warmup, 3)):
+    for i in range(args.warmup):
         _oracle_step(w, data, (i * 7 + 3) % nqt, 0)
+    # exactly K timed steps, each a bounded sample (one 128-row query tile of one head with
+    # that head's quantisation: 15-35 ms on 8-16 host cores, so K = 2000 takes about a minute)
     flops, t = 0.0, 0.0
-    steps = min(args.steps, 200)
+    steps = args.steps
     for i in range(steps):
         t0 = time.perf_counter()
         flops += _oracle_step(w, data, (i * 7 + 3) % nqt, (i * 5) % (w.B * w.Hq))
