@@ -58,6 +58,18 @@ MUTATIONS = [
     ("bf16 rounding ties away", "u += 0x7FFFu + ((u >> 16) & 1u);", "u += 0x8000u;"),
     ("bruteforce scale 1/d", "s[key] = acc / sqrt((double)d);", "s[key] = acc / (double)d;"),
     ("exact loop uses e^x", "P[kk] = valid[kk] ? exp2(S[kk] * cd - mnew64) : 0.0;", "P[kk] = valid[kk] ? exp(S[kk] * cd - mnew64) : 0.0;"),
+    ("rotated rows: smoothing divides", "v[i] = scale ? xv * scale[g * d + blk * 16 + i] : xv;\n            }\n            quant16(v, c, &scales[r * (d / 16) + blk]);\n            for (int i = 0; i < 8; ++i)\n                codes[r * (d / 2) + blk * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));\n        }\n    }\n}\n\n/* V^T", "v[i] = scale ? xv / scale[g * d + blk * 16 + i] : xv;\n            }\n            quant16(v, c, &scales[r * (d / 16) + blk]);\n            for (int i = 0; i < 8; ++i)\n                codes[r * (d / 2) + blk * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));\n        }\n    }\n}\n\n/* V^T"),
+    ("rotated rows: group index", "int g = h / grp;\n        const float* xr", "int g = h % Hkv;\n        const float* xr"),
+    ("two-level clamp -30", "if (p_t == 0.0f || k2 < -40) k2 = -40;", "if (p_t == 0.0f || k2 < -30) k2 = -30;"),
+    ("two-level without the clamp", "if (p_t == 0.0f || k2 < -40) k2 = -40;", "if (p_t == 0.0f) k2 = -40;"),
+    ("two-level L raised by k", "(double)(10 - e - k) - log2((double)(8 + m))", "(double)(10 - e + k) - log2((double)(8 + m))"),
+    ("two-level scale without 2^k", "float sigma = ldexpf(e4m3_value(sc), k2);", "float sigma = e4m3_value(sc);"),
+    ("causal loop skips the diagonal tile", "int ntiles = a->causal ? i / bc + 1 : N / bc;", "int ntiles = a->causal ? (i + 1) / bc : N / bc;"),
+    ("exact loop alpha sign", "double alpha = (mo == -INFINITY) ? 0.0 : exp2(mo - mn);", "double alpha = (mo == -INFINITY) ? 0.0 : exp2(mn - mo);"),
+    ("trace records P_hat as P", "out->tr_p[(j - jstart) * bc + kk] = (float)P[kk];", "out->tr_p[(j - jstart) * bc + kk] = (float)Ph[kk];"),
+    ("E2M1 magnitude 3 -> 2.5", "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f}", "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 2.5f, 4.0f, 6.0f}"),
+    ("merge O unweighted", "O[x] = fmaf(w, op[sp][x], O[x]);", "O[x] = op[sp][x] + O[x];"),
+    ("decode output off by one", "float inv = (L > 0.0f) ? 1.0f / L : 0.0f;", "float inv = (L > 0.0f) ? 1.0f / (L + 1.0f) : 0.0f;"),
 ]
 
 # one per area: formats, exp2, P_hat rule, block quantiser, packing, GEMM accumulation,

@@ -126,3 +126,41 @@ def test_closer_to_exact_attention(orc):
     print(f"\nrelative error vs fp64 attention: one level {rel(one):.4f}, two-level {rel(two):.4f}")
     assert rel(two) <= rel(one)
     assert rel(two) < 0.2
+
+
+def test_second_level_exponent_is_clamped_at_minus_40(orc):
+    # A tile far below the running max: k = max(floor(log2 p_t) - 10, -40) takes the clamp.
+    # Every query row is (6, 0, ..., 0) (Q_hat exact, scale 1); key n has K[n, 0] = kv[n]
+    # and zeros in channels 1..15, so S = 6 * kv[n] exactly (the K values -33, -42, -45
+    # quantise exactly, scales 5.5, 7, 7.5).  Keys outside kv tile 2 have S = 0 (m = 0).
+    # In tile 2 (keys 128..191, 64-key tiles): block A (S = -198: log2 P = -35.71) sets
+    # p_t, so floor(log2 p_t) - 10 = -46 and the clamp gives k = -40; blocks B and D
+    # (S = -252: log2 P = -45.45) keep a code (amax/6 * 2^40 = 0.0038 > 2^-10) and block C
+    # (S = -270: log2 P = -48.69) flushes (amax/6 * 2^40 = 0.0004 < 2^-10).  Without the
+    # clamp (k = -46) block C would keep a code; with a clamp at -30 blocks B and D would
+    # flush.  One level flushes the whole tile.
+    N, d, bc = 256, 64, 64
+    kv = np.zeros(N)
+    kv[128:144], kv[144:160], kv[160:176], kv[176:192] = -33.0, -42.0, -45.0, -42.0
+    q = np.zeros((N, d), np.float32)
+    q[:, 0] = 6.0
+    k = np.zeros((N, d), np.float32)
+    k[:, 0] = kv
+    rng = np.random.default_rng(65)
+    k[:, 16:] = rng.standard_normal((N, d - 16))
+    v = rng.standard_normal((N, d)).astype(np.float32)
+    bits = lambda a: gen.f32_to_bf16_bits(a)[None, None]
+    qz = orc.quantize_all(bits(q), bits(k), bits(v))
+    for row in (0, 200):
+        two = orc.attn_trace(qz, False, bc, row, two_level=True)
+        one = orc.attn_trace(qz, False, bc, row)
+        t2 = two["p"][2].astype(np.float64)
+        assert np.floor(np.log2(t2.max())) == -36
+        ph = two["phat"][2].reshape(4, 16)
+        assert np.all(ph[0] > 0) and np.all(ph[1] > 0) and np.all(ph[3] > 0), ph[:, 0]
+        assert np.all(ph[2] == 0), ph[:, 0]
+        assert np.all(one["phat"][2] == 0)
+        # the kept blocks are within the E2M1 bound of their scale sigma_b * 2^-40
+        for blk in (0, 1, 3):
+            p = t2[blk * 16:(blk + 1) * 16]
+            assert np.all(np.abs(ph[blk] - p) <= 0.36 * p)
