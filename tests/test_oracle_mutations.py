@@ -90,23 +90,46 @@ def _copy(dst):
 def _pins_pass(dst):
     tests = sorted(os.path.join("tests", f) for f in os.listdir(os.path.join(dst, "tests"))
                    if f.startswith("test_oracle_") and f != "test_oracle_mutations.py")
+    env = dict(os.environ, OMP_NUM_THREADS="2")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *tests],
-                       cwd=dst, capture_output=True, text=True, timeout=900)
+                       cwd=dst, capture_output=True, text=True, timeout=900, env=env)
     return r.returncode == 0, r.stdout[-2000:]
 
 
-def test_unmutated_copy_passes(tmp_path):
-    _copy(str(tmp_path))
-    ok, out = _pins_pass(str(tmp_path))
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    """{name: (pattern found once, pins pass, output tail)} for the unmutated copy
+    ("unmutated") and every selected mutation, run a few at a time."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    def work(job):
+        name, old, new = job
+        dst = str(tmp_path_factory.mktemp("mutant"))
+        _copy(dst)
+        found = True
+        if old is not None:
+            p = os.path.join(dst, SRC)
+            s = open(p).read()
+            found = s.count(old) == 1
+            if not found:
+                return name, (False, True, "")
+            open(p, "w").write(s.replace(old, new))
+        ok, out = _pins_pass(dst)
+        shutil.rmtree(dst, ignore_errors=True)
+        return name, (found, ok, out)
+
+    jobs = [("unmutated", None, None)] + SELECTED
+    with ThreadPoolExecutor(max_workers=max(1, min(4, (os.cpu_count() or 2) // 2))) as ex:
+        return dict(ex.map(work, jobs))
+
+
+def test_unmutated_copy_passes(outcomes):
+    found, ok, out = outcomes["unmutated"]
     assert ok, out
 
 
-@pytest.mark.parametrize("name,old,new", SELECTED, ids=[m[0] for m in SELECTED])
-def test_mutation_is_caught(tmp_path, name, old, new):
-    _copy(str(tmp_path))
-    p = os.path.join(str(tmp_path), SRC)
-    s = open(p).read()
-    assert s.count(old) == 1, f"the pattern of {name!r} no longer matches the oracle"
-    open(p, "w").write(s.replace(old, new))
-    ok, out = _pins_pass(str(tmp_path))
+@pytest.mark.parametrize("name", [m[0] for m in SELECTED])
+def test_mutation_is_caught(outcomes, name):
+    found, ok, _ = outcomes[name]
+    assert found, f"the pattern of {name!r} no longer matches the oracle"
     assert not ok, f"no pin fails when the oracle has: {name}"
