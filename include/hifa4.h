@@ -264,7 +264,9 @@ HIFA4_API int hifa4_attn_decode(const hifa4_qtensor* q, const hifa4_qtensor* k, 
 /*
  * The full attention forward on quantised Q, K and bf16 V: quantises V^T into
  * `workspace` (hifa4_attn_workspace_bytes(B, Hkv, N, d) bytes of device memory, 16-byte
- * aligned), then runs hifa4_attn_fwd_quantized.  Two launches on `stream`.
+ * aligned), then runs hifa4_attn_fwd_quantized.  Two launches on `stream`.  Every
+ * argument, those of the attention included, is checked before the first launch: an
+ * error status means nothing was enqueued.
  */
 HIFA4_API size_t hifa4_attn_workspace_bytes(int B, int Hkv, int N, int d);
 HIFA4_API int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v, const int64_t v_strides[3],
