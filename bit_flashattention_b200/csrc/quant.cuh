@@ -3,8 +3,8 @@
 // tokens per channel), and the per-channel amax reduction of the Smooth-QK calibration.
 //
 // Smooth-QK ("HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs for LLM
-// Inference", abstract): a calibration-static per-channel equivalent rescaling Q*s, K/s
-// after RoPE, with no per-tile online reduction at inference.  Here q' = RN(q * s[g,c])
+// Inference", abstract): after RoPE, Q is multiplied and K divided per channel by scales s
+// that an offline calibration fixes, so inference computes no statistics for it.  Here q' = RN(q * s[g,c])
 // and k' = RN(k * s_inv[g,c]) with g the kv head of the query head.
 #pragma once
 #include "method.cuh"

@@ -13,8 +13,8 @@ Recipe (per workload, see ``configs.py``):
     and K when the workload has a RoPE base.
   * Then, on K only: the seeded outlier channels of each kv head are multiplied by the
     outlier factor, and a per-(kv head, channel) bias ~ N(0, 1) is added when enabled.
-    Smooth-QK is calibrated on and applied to these post-RoPE tensors (HiFA4 abstract:
-    "per-channel equivalent rescaling to Q and K after RoPE").
+    Smooth-QK is calibrated on and applied to these post-RoPE tensors (the HiFA4
+    abstract applies its per-channel scales after RoPE).
   * Everything is rounded to bf16 (round to nearest even) and returned as uint16 bits.
 
 The pages measure on MMLU traces of real models; those are not available here, so these

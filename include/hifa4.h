@@ -98,8 +98,8 @@ HIFA4_API size_t hifa4_qtensor_codes_bytes(int B, int H, int N, int d);
 HIFA4_API size_t hifa4_qtensor_scales_bytes(int B, int H, int N, int d, int transposed);
 
 /*
- * Smooth-QK calibration (HiFA4 abstract: "calibration-static per-channel equivalent
- * rescaling to Q and K after RoPE").  From a post-RoPE bf16 calibration sample Q_cal
+ * Smooth-QK calibration (HiFA4 abstract: per-channel scales for post-RoPE Q and K, fixed
+ * offline from a calibration sample).  From a post-RoPE bf16 calibration sample Q_cal
  * [B, Hq, N, d] and K_cal [B, Hkv, N, d]:
  *   s[g, c]    = RN_fp32((amax_K[g, c] / amax_Q[g, c]) ^ alpha), computed in double
  *                (s = 1 where either amax is 0; alpha = 0 gives s == 1),
@@ -204,10 +204,10 @@ HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtens
  * chunks in order).
  *   normaliser 0: l from r = P_hat * 1 as in HiFA4 (O, m, l identical to
  *                 hifa4_attn_fwd_quantized);
- *   normaliser 1: l from r = sum P, the "inconsistent formulation" of the HiFA4 abstract
+ *   normaliser 1: l from r = sum P, the inconsistent formulation of the HiFA4 abstract
  *                 (PV still uses P_hat), i.e. each tile's contribution to O is scaled by
  *                 sum P_hat / sum P.  With Q and K quantised without Smooth-QK (s = NULL)
- *                 this is the abstract's "direct HIF4 quantization" baseline.
+ *                 this is the abstract's baseline of direct 4-bit quantisation.
  *   two_level 0: the one-level block scales of P_hat (as hifa4_attn_fwd_quantized);
  *   two_level 1: a second-level scale for P: per row and kv tile a power of two 2^k,
  *                k = max(floor(log2 p_t) - 10, -40) with p_t the tile's largest block amax

@@ -11,8 +11,8 @@
  * Source of the method: "HiFA4: Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs
  * for LLM Inference" (abstract, as printed on catalyzex.com/author/Chunlu Li, the same
  * text on the other pages).  The abstract fixes: both QK^T and PV are 4-bit GEMMs; the
- * online-softmax state is FP16; Smooth-QK is a calibration-static per-channel rescaling
- * Q*s, K/s applied after RoPE; P-Reordering sums the normaliser from the same quantised
+ * online-softmax state is FP16; Smooth-QK multiplies Q and divides K per channel by
+ * scales s that an offline calibration fixes, after RoPE; P-Reordering sums the normaliser from the same quantised
  * weights P_hat that feed PV, which lets the normaliser be produced by the PV GEMM.
  * Everything the abstract leaves open is a stated reading (listed in the design notes):
  *   - 4-bit format: E2M1 values with one unsigned E4M3 scale per 16 contraction
