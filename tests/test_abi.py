@@ -148,3 +148,15 @@ def test_rope_table_matches_float64_angles():
         assert np.all(np.abs(got.astype(np.float64) - ref) <= 0.5 * ulp + 1e-12)
     with pytest.raises(hifa4.Hifa4Error):
         hifa4.hifa4_rope_table(1.0, N, d)
+
+
+def test_product_path_fails_loudly_without_the_library(monkeypatch):
+    # no CPU fallback: with libhifa4.so absent every entry point raises instead of computing
+    monkeypatch.setattr(hifa4, "LIB_PATH", "/nonexistent/libhifa4.so")
+    monkeypatch.setattr(hifa4, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        hifa4.lib()
+    with pytest.raises(RuntimeError, match="missing"):
+        hifa4.QTensor(1, 1, 128, 128, 0, "cuda")
+    with pytest.raises(RuntimeError, match="missing"):
+        hifa4.status_string(0)
