@@ -160,3 +160,37 @@ def test_product_path_fails_loudly_without_the_library(monkeypatch):
         hifa4.QTensor(1, 1, 128, 128, 0, "cuda")
     with pytest.raises(RuntimeError, match="missing"):
         hifa4.status_string(0)
+
+
+def test_empty_and_degenerate_shapes_are_rejected_on_the_host(L):
+    # zero batch, heads, tokens or query tokens, and head counts that do not divide, are
+    # refused before any device work (on a machine without a GPU a launch attempt would
+    # report UNSUPPORTED_DEVICE instead)
+    buf = np.zeros(1 << 16, np.uint8)
+    p = ctypes.c_void_p(((buf.ctypes.data + 15) // 16) * 16)
+    status = ctypes.c_void_p(p.value + 32768)
+    st = (ctypes.c_int64 * 3)(0, 0, 128)
+    SHAPE = hifa4.ERR_UNSUPPORTED_SHAPE
+    for B, H, N in ((0, 1, 128), (1, 0, 128), (1, 1, 0)):
+        qt = hifa4._QT(p, p, B, H, N, 128, 0)
+        vt = hifa4._QT(p, p, B, H, N, 128, 1)
+        assert L.hifa4_quantize_qk(p, p, st, st, B, H, H if H else 1, N, 128, None, None, ctypes.byref(qt),
+                                   ctypes.byref(qt), status, None) == SHAPE
+        assert L.hifa4_quantize_v(p, st, B, H, N, 128, ctypes.byref(vt), status, None) == SHAPE
+        assert L.hifa4_quantize_qkv(p, p, p, st, st, st, B, H, H if H else 1, N, 128, None, None, ctypes.byref(qt),
+                                    ctypes.byref(qt), ctypes.byref(vt), status, None) == SHAPE
+        assert L.hifa4_attn_fwd_quantized(ctypes.byref(qt), ctypes.byref(qt), ctypes.byref(vt), B, H, H if H else 1,
+                                          N, 128, 1, 0, p, None, None, status, None) == SHAPE
+    ws = ctypes.c_size_t(1 << 15)
+    q = hifa4._QT(p, p, 1, 1, 128, 128, 0)
+    for nq, Nk in ((0, 256), (1, 0), (129, 256)):
+        k = hifa4._QT(p, p, 1, 1, Nk, 128, 0)
+        v = hifa4._QT(p, p, 1, 1, Nk, 128, 1)
+        assert L.hifa4_attn_decode(ctypes.byref(q), ctypes.byref(k), ctypes.byref(v), 1, 1, 1, nq, Nk, 128, 0, 0, p,
+                                   ws, p, None, None, status, None) == SHAPE
+    assert L.hifa4_calibrate_smooth(p, p, st, st, 1, 1, 1, 0, 128, 0.5, p, p, p, None) == SHAPE
+    assert L.hifa4_calibrate_smooth(p, p, st, st, 1, 3, 2, 16, 128, 0.5, p, p, p, None) == SHAPE
+    assert L.hifa4_calibrate_smooth(p, p, st, st, 1, 1, 1, 16, 128, -0.5, p, p, p, None) == hifa4.ERR_INVALID_ARG
+    # size helpers give 0 for empty tensors
+    assert L.hifa4_qtensor_codes_bytes(0, 1, 128, 128) == 0 and L.hifa4_qtensor_scales_bytes(1, 1, 0, 128, 0) == 0
+    assert L.hifa4_decode_workspace_bytes(1, 1, 0, 128) == 0 and L.hifa4_decode_workspace_bytes(1, 1, 65, 128) == 0
