@@ -5,7 +5,7 @@ import numpy as np
 import torch
 
 import oracle
-from bit_flashattention_b200 import configs, gen, hifa4
+from bit_flashattention_b200 import gen, hifa4
 from tests import _layout
 
 # Tolerances on the attention output O (per the target: FP16 m and l exact, codes and

@@ -4,7 +4,6 @@ probes of the block-scaled FP4 tensor-core MMAs (the S accumulation probe fixes 
 fp32 accumulation model the oracle mirrors)."""
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from bit_flashattention_b200 import configs, gen, hifa4

@@ -2,7 +2,6 @@
 4-bit dot product (S) against library routines, invariants and closed forms."""
 import ml_dtypes
 import numpy as np
-import pytest
 
 from bit_flashattention_b200 import configs, gen
 

@@ -6,7 +6,6 @@ must give what hifa4_attn_fwd gives on the same inputs, and it must reject a wor
 whose scratch would not fit.  Collected last so that a failure here cannot hide others."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
