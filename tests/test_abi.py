@@ -194,3 +194,26 @@ def test_empty_and_degenerate_shapes_are_rejected_on_the_host(L):
     # size helpers give 0 for empty tensors
     assert L.hifa4_qtensor_codes_bytes(0, 1, 128, 128) == 0 and L.hifa4_qtensor_scales_bytes(1, 1, 0, 128, 0) == 0
     assert L.hifa4_decode_workspace_bytes(1, 1, 0, 128) == 0 and L.hifa4_decode_workspace_bytes(1, 1, 65, 128) == 0
+
+
+def test_header_is_plain_c_and_a_c_program_links(L, tmp_path):
+    # include/hifa4.h is a C header (no torch or C++ types): a C11 program includes it,
+    # links against libhifa4.so and calls a host-only entry point
+    import os
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.join(root, "bit_flashattention_b200")
+    src = tmp_path / "use_hifa4.c"
+    src.write_text('#include "hifa4.h"\n'
+                   'int main(void) {\n'
+                   '  if (hifa4_qtensor_codes_bytes(1, 2, 128, 64) != 8192) return 1;\n'
+                   '  if (hifa4_qtensor_scales_bytes(1, 2, 128, 64, 0) != 1024) return 2;\n'
+                   '  return hifa4_status_string(HIFA4_ERR_TIMEOUT)[0] == \'H\' ? 0 : 3;\n'
+                   '}\n')
+    exe = tmp_path / "use_hifa4"
+    cuda_inc = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "include")
+    r = subprocess.run(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(root, "include"), "-I", cuda_inc,
+                        str(src), "-o", str(exe), "-L", libdir, "-lhifa4", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert subprocess.run([str(exe)]).returncode == 0
