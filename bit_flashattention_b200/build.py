@@ -6,7 +6,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRCS = [os.path.join(HERE, "csrc", f) for f in ("hifa4_api.cu", "hifa4_noalloc.cu")]
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("ptx.cuh", "method.cuh", "quant.cuh", "attn.cuh")] + \
+# every header the two translation units include: a change to any of them rebuilds
+DEPS = sorted(os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc")) if f.endswith(".cuh")) + \
        [os.path.join(ROOT, "include", "hifa4.h")]
 LIB = os.path.join(HERE, "libhifa4.so")
 
