@@ -158,3 +158,42 @@ def test_s_dot_rz_model_against_integer_arithmetic(orc):
                         t += isum * sc(int(qs[i, b])) * sc(int(ks[k, b]))
                     acc = _rz_f32(int(round(acc * 2 ** 20)) + t, 20)
                 assert got[i, k] == np.float32(acc)
+
+
+def test_smooth_qk_leaves_qkt_unchanged_in_exact_arithmetic(orc):
+    # (Q*s)(K/s)^T = QK^T.  Exactly representable case: s constant over each 16-channel
+    # block and a power of two, so Q*s and K/s are exact, each block's codes are unchanged
+    # and its E4M3 scale moves by the same power of two in opposite directions (scales stay
+    # normal here); the exact 4-bit dot products, and so the whole quantised attention,
+    # must then be bit-identical with and without Smooth-QK.
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=4, Hkv=2, N=256, d=128, bc=64)
+    q, k, v = gen.inputs(w)
+    rng = np.random.default_rng(10)
+    e = rng.integers(-2, 3, (w.Hkv, w.d // 16))
+    s = np.repeat(np.float32(2.0) ** e.astype(np.float32), 16, axis=1)
+    sinv = (np.float32(1.0) / s).astype(np.float32)
+    plain = orc.quantize_all(q, k, v)
+    smooth = orc.quantize_all(q, k, v, s, sinv)
+    assert np.array_equal(plain.qc, smooth.qc) and np.array_equal(plain.kc, smooth.kc)
+    g = np.repeat(np.arange(w.Hkv), w.Hq // w.Hkv)
+    assert np.array_equal(smooth.qs.astype(int) - plain.qs.astype(int), np.broadcast_to(8 * e[g][None, :, None, :],
+                                                                                          plain.qs.shape))
+    assert np.array_equal(smooth.ks.astype(int) - plain.ks.astype(int), np.broadcast_to(-8 * e[None, :, None, :],
+                                                                                          plain.ks.shape))
+    for h in range(w.Hq):
+        S0 = orc.qk_scores(plain.qc[0, h], plain.qs[0, h], plain.kc[0, g[h]], plain.ks[0, g[h]], 2)
+        S1 = orc.qk_scores(smooth.qc[0, h], smooth.qs[0, h], smooth.kc[0, g[h]], smooth.ks[0, g[h]], 2)
+        assert np.array_equal(S0, S1)
+    a, b = orc.attn_fwd(plain, True, w.bc), orc.attn_fwd(smooth, True, w.bc)
+    assert all(np.array_equal(a[x], b[x]) for x in ("o_bf16", "m", "l"))
+    # and with the calibrated (not power-of-two) s, fp64 (Q*s)(K*s_inv)^T stays within the
+    # rounding of s_inv = RN(1/s) of QK^T
+    qc, kc, _ = gen.inputs(w, calib=True)
+    sc, sci = orc.calibrate(qc, kc, 0.5)
+    qf = gen.bf16_bits_to_f32(q).astype(np.float64)[0]
+    kf = gen.bf16_bits_to_f32(k).astype(np.float64)[0]
+    for h in range(w.Hq):
+        ref = qf[h] @ kf[g[h]].T
+        got = (qf[h] * sc[g[h]]) @ (kf[g[h]] * sci[g[h]]).T
+        bound = np.abs(qf[h]) @ np.abs(kf[g[h]]).T * 2.0 ** -23
+        assert np.all(np.abs(got - ref) <= bound)
