@@ -14,27 +14,27 @@
  * online-softmax state is FP16; Smooth-QK multiplies Q and divides K per channel by
  * scales s that an offline calibration fixes, after RoPE; P-Reordering sums the normaliser from the same quantised
  * weights P_hat that feed PV, which lets the normaliser be produced by the PV GEMM.
- * Everything the abstract leaves open is a stated reading (listed in the design notes):
+ * Everything the abstract leaves open is a stated reading:
  *   - 4-bit format: E2M1 values with one unsigned E4M3 scale per 16 contraction
  *     elements (NVFP4-style), no second-level scale.  scale = E4M3_RN(amax * RN(1/6)),
  *     R = RN(1/scale) (R = 0 when scale == 0), code = E2M1_RN_satfinite(x * R).
  *   - exp2 in the softmax: the method's own deterministic approximation E(x) (clamp to
- *     -127, floor split, quadratic Horner in fp32 fma, exponent insert); see own_exp2().
+ *     -127, floor split, cubic Horner in fp32 fma, exponent insert; relative error below
+ *     9e-5); see own_exp2().
  *   - m_new = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e)/sqrt(d)),
  *     P = E(RN(fma(S, c, -m_new))), alpha = E(RN(m_old - m_new)),
- *     a block's scale sigma comes from E(fma(blockmax(S), c, -m_new)) (equal to the block
- *     amax of P because E is monotone -- pinned by a test), and a score's P_hat code is
- *     the E2M1 rounding of P/sigma evaluated in the log domain with a linear mantissa
- *     (phat_value()),
+ *     P_hat = the block quantiser above applied to P, 16 consecutive keys per block
+ *     (so a score's code is E2M1_RN(RN(P * RN(1/sigma))) with sigma from the block's
+ *     largest P),
  *     l = fp16_RN(fma(alpha, l, r)), r = exact sum of the tile's P_hat,
  *     O = alpha*O (fp32) + (exact tile P_hat V_hat rounded to fp32),
  *     out = bf16_RN(RN(O / l)).
  *   - two-level P scale (ablation variant, two_level = 1): a per-(row, tile) power of two
  *     2^k under the block scales of P, k = max(floor(log2 p_t) - 10, -40) with p_t the
  *     tile's largest block amax of P; sigma_b = E4M3_RN(RN(amax * RN(1/6)) * 2^-k),
- *     P_hat = code * sigma_b * 2^k, L from the effective scale sigma_b * 2^k.  Where the
- *     one-level scale is a normal E4M3 value both give the same P_hat; blocks too small
- *     for one level (scale 0 or subnormal) keep their mass.
+ *     P_hat = code * sigma_b * 2^k with code = E2M1_RN(RN(P * RN(1/(sigma_b * 2^k)))).
+ *     Where the one-level scale is a normal E4M3 value both give the same P_hat; blocks
+ *     too small for one level (scale 0 or subnormal) keep their mass.
  *   - S accumulation of the 4-bit GEMM: one of the models in s_dot(), selected by the
  *     caller; the mirror uses model 3 (per 64-wide MMA step, the exact sum of the fp32
  *     accumulator and the step's block products, rounded toward zero), which is what a
@@ -133,75 +133,37 @@ static uint8_t e4m3_encode_pos(float x) {
 
 /* ------------------------------------------------------------------ own exp2 E(x) */
 
-/* Coefficients of p(f) = 1 + c1 f + c2 f^2 ~ 2^f on [0,1): a minimax fit of the relative
- * error with p(0) = 1 held exact (max relative error 2.05e-3, far below the spacing of the
- * 4-bit codes P is rounded to), rounded to fp32. */
-#define EXP2_C1 0x1.54f8d6p-1f
-#define EXP2_C2 0x1.51d9ccp-2f
+/* Coefficients of p(f) = 1 + c1 f + c2 f^2 + c3 f^3 ~ 2^f on [0,1): a minimax fit of the
+ * relative error with p(0) = 1 held exact (max relative error 8.6e-5), rounded to fp32. */
+#define EXP2_C1 0x1.63e65ap-1f
+#define EXP2_C2 0x1.d23788p-3f
+#define EXP2_C3 0x1.3baaa8p-4f
 
 static float own_exp2(float x) {
     float xc = fmaxf(x, -127.0f);            /* fmaxf(NaN,-127) = -127; -inf -> -127 */
     float n = floorf(xc);
-    float f = xc - n;                        /* exact */
-    float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);
+    float f = xc - n;                        /* RN(xc - n) */
+    float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);
     uint32_t bits = f32_bits(p) + ((uint32_t)(int32_t)n << 23);
     return bits_f32(bits);                   /* p * 2^n; exactly 0 for xc = -127 */
 }
 
-/* ------------------------------------------------------------------ P_hat codes */
-
-/* L(sigma) = RN_fp32(-log2(sigma)) of a positive E4M3 scale, from its integer parts:
- * normal sigma = (8 + m) * 2^(e - 10) gives (10 - e) - log2(8 + m); subnormal
- * sigma = m * 2^-9 gives 9 - log2(m); each computed in double, rounded once to fp32. */
-static float neg_log2_scale(uint8_t code) {
-    int e = (code >> 3) & 15, m = code & 7;
-    double v = (e == 0) ? 9.0 - log2((double)m) : (double)(10 - e) - log2((double)(8 + m));
-    return (float)v;
-}
-
-/* L of the effective scale sigma * 2^k (two-level P scale): the same integer-log form with
- * the integer part lowered by k before the one subtraction, so k = 0 is neg_log2_scale. */
-static float neg_log2_scale_k(uint8_t code, int k) {
-    int e = (code >> 3) & 15, m = code & 7;
-    double v = (e == 0) ? (double)(9 - k) - log2((double)m) : (double)(10 - e - k) - log2((double)(8 + m));
-    return (float)v;
-}
-
-/* The value whose E2M1 rounding is the P_hat code of a score: P / sigma evaluated in the
- * log domain with a linear mantissa.  Per block, B = RN(RN(L(sigma) - m) + 125) / 128;
- * per score
- *   u = min(1, max(0, RN(S * (c/128) + B)))          (NaN -> 0)
- *   z = 128 u - 125 + DELTA, rounded to a multiple of 2^-10 (round to nearest even)
- *   y = 2^floor(z) * (1 + z - floor(z)).
- * 128 u - 125 is log2(P / sigma) = S c - m - log2(sigma) held in [-125, 3]; y is the
- * piecewise-linear (linear-mantissa) exponential of z.  Only the E2M1 code of y is used,
- * and that code changes where y crosses 0.25, 0.75, 1.25, 1.75, 2.5, 3.5 and 5: with
- * DELTA = -73/1024 those crossings lie within 0.014 (log2 units) of the crossings of the
- * exact 2^(S c - m) / sigma, except the crossing at 0.25 (codes 0 and 1), which lies 0.071
- * above it.  Outside [-125, 3] every code is already 0 or saturated. */
-#define PHAT_DELTA (-73.0 / 1024.0)
-static float phat_value(float S, float c, float B) {
-    float u = fmaf(S, c * 0.0078125f, B);
-    if (!(u > 0.0f)) u = 0.0f;
-    if (u > 1.0f) u = 1.0f;
-    double t = (double)u * 128.0 - 125.0 + PHAT_DELTA;   /* exact: u has 24 bits */
-    double z = nearbyint(t * 1024.0) / 1024.0;           /* round half to even */
-    double k = floor(z);
-    return (float)ldexp(1.0 + (z - k), (int)k);          /* exact: 11 significant bits */
-}
-
 /* ------------------------------------------------------------------ block quantiser */
 
-/* NVFP4-style block of 16: scale from the amax, codes from x * (1/scale). */
-static void quant16(const float* x, uint8_t* codes /*16 nibbles, one per byte*/, uint8_t* scale) {
+/* NVFP4-style block of 16 with an optional second-level power of two 2^k (k = 0: the
+ * one-level format): the E4M3 scale is taken of RN(amax * RN(1/6)) * 2^-k, the effective
+ * scale is sigma = scale * 2^k, and every code is E2M1_RN(RN(x * RN(1/sigma))). */
+static void quant16_k(const float* x, int k, uint8_t* codes /*16 nibbles, one per byte*/, uint8_t* scale) {
     float amax = 0.0f;
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    uint8_t sc = e4m3_encode_pos(amax * (1.0f / 6.0f));
-    float sigma = e4m3_value(sc);
+    uint8_t sc = e4m3_encode_pos(ldexpf(amax * (1.0f / 6.0f), -k));
+    float sigma = ldexpf(e4m3_value(sc), k);
     float R = (sigma == 0.0f) ? 0.0f : 1.0f / sigma;
     for (int i = 0; i < 16; ++i) codes[i] = e2m1_encode(x[i] * R);
     *scale = sc;
 }
+
+static void quant16(const float* x, uint8_t* codes, uint8_t* scale) { quant16_k(x, 0, codes, scale); }
 
 /* ------------------------------------------------------------------ exported codec */
 
@@ -526,13 +488,12 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
         double P[256], Ph[256];
         for (int kk = 0; kk < bc; ++kk) { P[kk] = 0.0; Ph[kk] = 0.0; }
         if (a->quant) {
-            float amaxs[16];
-            float p_t = 0.0f;                                 /* the tile's largest block amax */
-            for (int blk = 0; blk < bc / 16; ++blk) {
-                float bmax = -INFINITY;
-                for (int e = 0; e < 16; ++e) bmax = fmaxf(bmax, Sf[blk * 16 + e]);
-                amaxs[blk] = own_exp2(fmaf(bmax, c, -mref));  /* = block amax of P (E monotone) */
-                if (amaxs[blk] > p_t) p_t = amaxs[blk];
+            /* P of every key (masked keys: S = -inf gives P = 0) */
+            float Pf[256];
+            float p_t = 0.0f;                                 /* the tile's largest P */
+            for (int kk = 0; kk < bc; ++kk) {
+                Pf[kk] = own_exp2(fmaf(Sf[kk], c, -mref));
+                if (Pf[kk] > p_t) p_t = Pf[kk];
             }
             int k2 = 0;                                       /* second-level scale 2^k2 */
             if (a->two_level) {
@@ -541,18 +502,15 @@ static void row_loop(const loop_args* a, long long row, row_out* out) {
                 k2 = (ex - 1) - 10;
                 if (p_t == 0.0f || k2 < -40) k2 = -40;
             }
+            /* P_hat: the block quantiser on each 16 consecutive keys of P */
             for (int blk = 0; blk < bc / 16; ++blk) {
-                float amax = amaxs[blk];
-                uint8_t sc = e4m3_encode_pos(ldexpf(amax * (1.0f / 6.0f), -k2));
+                uint8_t code[16], sc;
+                quant16_k(Pf + blk * 16, k2, code, &sc);
                 float sigma = ldexpf(e4m3_value(sc), k2);
-                float B = -INFINITY;                          /* sigma == 0: every code is 0 */
-                if (sigma > 0.0f) B = ((neg_log2_scale_k(sc, k2) - mref) + 125.0f) * 0.0078125f;
                 for (int e = 0; e < 16; ++e) {
                     int kk = blk * 16 + e;
-                    float p = own_exp2(fmaf(Sf[kk], c, -mref));
-                    uint8_t code = e2m1_encode(phat_value(Sf[kk], c, B));
-                    P[kk] = p;
-                    Ph[kk] = (double)e2m1_value(code) * sigma;
+                    P[kk] = Pf[kk];
+                    Ph[kk] = (double)e2m1_value(code[e]) * sigma;
                 }
             }
         } else {
@@ -788,12 +746,6 @@ OR_EXPORT int or_attn_bruteforce(const uint16_t* q, const uint16_t* k, const uin
 }
 
 OR_EXPORT uint16_t or_f16_bits(float f) { return f16_bits(f); }
-
-OR_EXPORT float or_neg_log2_scale(uint8_t code) { return neg_log2_scale(code); }
-
-OR_EXPORT void or_phat_values(const float* S, size_t n, float c, float B, float* y) {
-    for (size_t i = 0; i < n; ++i) y[i] = phat_value(S[i], c, B);
-}
 
 OR_EXPORT int or_num_threads(void) {
 #ifdef _OPENMP

@@ -69,9 +69,6 @@ def lib():
         L.or_f16_bits.argtypes = [ctypes.c_float]
         L.or_f16_bits.restype = ctypes.c_uint16
         L.or_num_threads.restype = i
-        L.or_neg_log2_scale.argtypes = [ctypes.c_uint8]
-        L.or_neg_log2_scale.restype = ctypes.c_float
-        L.or_phat_values.argtypes = [P, sz, ctypes.c_float, ctypes.c_float, P]
         _lib = L
     return _lib
 
@@ -126,17 +123,6 @@ def quant_blocks(x):
     scales = np.empty(x.size // 16, np.uint8)
     lib().or_quant_blocks(_p(x), x.size, _p(codes), _p(scales))
     return codes, scales
-
-
-def neg_log2_scale(code: int) -> float:
-    return lib().or_neg_log2_scale(code)
-
-
-def phat_values(S, c, B):
-    S = _c(S, np.float32)
-    y = np.empty(S.shape, np.float32)
-    lib().or_phat_values(_p(S), S.size, float(c), float(B), _p(y))
-    return y
 
 
 def f16_bits(x: float) -> int:

@@ -22,12 +22,20 @@ MUTATIONS = [
     ("e4m3 ties to odd", "return (uint8_t)((lo & 1) ? hi : lo);", "return (uint8_t)((lo & 1) ? lo : hi);"),
     ("e4m3 saturates to NaN", "if (x >= 448.0f) return 0x7E;", "if (x >= 448.0f) return 0x7F;"),
     ("exp2 clamp -126", "float xc = fmaxf(x, -127.0f);", "float xc = fmaxf(x, -126.0f);"),
-    ("exp2 coefficient c1", "#define EXP2_C1 0x1.54f8d6p-1f", "#define EXP2_C1 0x1.56f8d6p-1f"),
-    ("exp2 drops the quadratic term", "float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);", "float p = fmaf(EXP2_C1, f, 1.0f);"),
-    ("L(sigma) exponent offset", "(double)(10 - e) - log2((double)(8 + m));\n    return (float)v;\n}\n\n/* L of the effective", "(double)(9 - e) - log2((double)(8 + m));\n    return (float)v;\n}\n\n/* L of the effective"),
-    ("phat delta sign", "#define PHAT_DELTA (-73.0 / 1024.0)", "#define PHAT_DELTA (73.0 / 1024.0)"),
-    ("phat offset 124", "double t = (double)u * 128.0 - 125.0 + PHAT_DELTA;", "double t = (double)u * 128.0 - 124.0 + PHAT_DELTA;"),
-    ("block scale 1/4", "uint8_t sc = e4m3_encode_pos(amax * (1.0f / 6.0f));", "uint8_t sc = e4m3_encode_pos(amax * (1.0f / 4.0f));"),
+    ("exp2 coefficient c1", "#define EXP2_C1 0x1.63e65ap-1f", "#define EXP2_C1 0x1.65e65ap-1f"),
+    ("exp2 drops the cubic term", "float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);",
+     "float p = fmaf(fmaf(EXP2_C2, f, EXP2_C1), f, 1.0f);"),
+    ("exp2 quadratic fit", "float p = fmaf(fmaf(fmaf(EXP2_C3, f, EXP2_C2), f, EXP2_C1), f, 1.0f);",
+     "float p = fmaf(fmaf(0x1.51d9ccp-2f, f, 0x1.54f8d6p-1f), f, 1.0f);"),
+    ("linear-mantissa P_hat", "float sigma = ldexpf(e4m3_value(sc), k2);\n",
+     "float sigma = ldexpf(e4m3_value(sc), k2);\n"
+     "                for (int e = 0; e < 16; ++e) {\n"
+     "                    double pr = Pf[blk * 16 + e];\n"
+     "                    if (!(pr > 0.0) || !(sigma > 0.0f)) { code[e] = 0; continue; }\n"
+     "                    double z = log2(pr / sigma) - 73.0 / 1024.0, fl = floor(z);\n"
+     "                    code[e] = e2m1_encode((float)ldexp(1.0 + (z - fl), (int)fl));\n"
+     "                }\n"),
+    ("block scale 1/4", "uint8_t sc = e4m3_encode_pos(ldexpf(amax * (1.0f / 6.0f), -k));", "uint8_t sc = e4m3_encode_pos(ldexpf(amax * (1.0f / 4.0f), -k));"),
     ("block R halved", "float R = (sigma == 0.0f) ? 0.0f : 1.0f / sigma;", "float R = (sigma == 0.0f) ? 0.0f : 0.5f / sigma;"),
     ("row packing nibble order", "codes[r * (d / 2) + blk * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));\n        }\n    }\n}\n\n/* Rotate-half", "codes[r * (d / 2) + blk * 8 + i] = (uint8_t)(c[2 * i + 1] | (c[2 * i] << 4));\n        }\n    }\n}\n\n/* Rotate-half"),
     ("row quantiser group index", "int g = h / grp;\n        const uint16_t* xr", "int g = h % Hkv;\n        const uint16_t* xr"),
@@ -43,7 +51,8 @@ MUTATIONS = [
     ("l not rescaled", "l16 = f16_round(fmaf(alpha, l16, (float)r));", "l16 = f16_round(fmaf(1.0f, l16, (float)r));"),
     ("normaliser from P (not P_hat)", "r += a->l_from_p ? P[kk] : Ph[kk];", "r += a->l_from_p ? Ph[kk] : P[kk];"),
     ("epilogue off by one", "float o = O32[x] / l16;", "float o = O32[x] / (l16 + 1.0f);"),
-    ("block scale ignores m", "amaxs[blk] = own_exp2(fmaf(bmax, c, -mref));", "amaxs[blk] = own_exp2(fmaf(bmax, c, 0.0f));"),
+    ("P ignores m", "Pf[kk] = own_exp2(fmaf(Sf[kk], c, -mref));", "Pf[kk] = own_exp2(fmaf(Sf[kk], c, 0.0f));"),
+    ("two-level R without 2^-k", "float sigma = ldexpf(e4m3_value(sc), k);", "float sigma = e4m3_value(sc);"),
     ("GQA kv head index", "const int g = h / (a->Hq / a->Hkv);", "const int g = h % a->Hkv;"),
     ("V scale of the next block", "e4m3_value(a->vs[vr * (Nk / 16) + key / 16]);", "e4m3_value(a->vs[vr * (Nk / 16) + (key / 16 + 1) % (Nk / 16)]);"),
     ("O accumulation drops half of PV", "O32[x] = (float)((double)O32[x] + pv[x]);", "O32[x] = (float)((double)O32[x] + 0.5 * pv[x]);"),
@@ -62,7 +71,6 @@ MUTATIONS = [
     ("rotated rows: group index", "int g = h / grp;\n        const float* xr", "int g = h % Hkv;\n        const float* xr"),
     ("two-level clamp -30", "if (p_t == 0.0f || k2 < -40) k2 = -40;", "if (p_t == 0.0f || k2 < -30) k2 = -30;"),
     ("two-level without the clamp", "if (p_t == 0.0f || k2 < -40) k2 = -40;", "if (p_t == 0.0f) k2 = -40;"),
-    ("two-level L raised by k", "(double)(10 - e - k) - log2((double)(8 + m))", "(double)(10 - e + k) - log2((double)(8 + m))"),
     ("two-level scale without 2^k", "float sigma = ldexpf(e4m3_value(sc), k2);", "float sigma = e4m3_value(sc);"),
     ("causal loop skips the diagonal tile", "int ntiles = a->causal ? i / bc + 1 : N / bc;", "int ntiles = a->causal ? (i + 1) / bc : N / bc;"),
     ("exact loop alpha sign", "double alpha = (mo == -INFINITY) ? 0.0 : exp2(mo - mn);", "double alpha = (mo == -INFINITY) ? 0.0 : exp2(mn - mo);"),
@@ -74,7 +82,7 @@ MUTATIONS = [
 
 # one per area: formats, exp2, P_hat rule, block quantiser, packing, GEMM accumulation,
 # running max, normaliser, merge, calibration, output rounding
-DEFAULT = {"e4m3 ties to odd", "exp2 drops the quadratic term", "phat delta sign", "block R halved",
+DEFAULT = {"e4m3 ties to odd", "exp2 quadratic fit", "linear-mantissa P_hat", "block R halved",
            "row packing nibble order", "S accumulation RN instead of RZ", "m not rounded to fp16",
            "normaliser from P (not P_hat)", "merge weight sign", "calibration ratio inverted",
            "bf16 rounding ties away"}
@@ -119,6 +127,7 @@ def outcomes(tmp_path_factory):
         return name, (found, ok, out)
 
     jobs = [("unmutated", None, None)] + SELECTED
+    tmp_path_factory.getbasetemp()            # create the base directory before the threads do
     with ThreadPoolExecutor(max_workers=max(1, min(4, (os.cpu_count() or 2) // 2))) as ex:
         return dict(ex.map(work, jobs))
 
