@@ -57,7 +57,7 @@ struct AttnCfg {
   static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
   static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
-  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 128 x fp32 table of L(sigma)
+  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;            // 256 x fp32: RN(1/sigma) (fast rule: L(sigma))
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 1024;          // [2][NSW][128] fp32 partial row maxima
   static constexpr uint32_t OFF_XSUM = OFF_XMAX + 2 * 4 * 128 * 4;   // [2][NSW][128] partial sums of P (ablation)
   static constexpr uint32_t OFF_BAR = OFF_XSUM + 2 * 4 * 128 * 4;
@@ -115,8 +115,7 @@ struct AttnParams {
   // block scales of P, k = max(floor(log2 p_t) - 10, -40), p_t the tile's largest block
   // amax; TMEM then holds O * 2^-k and R * 2^-k
   int two_level;
-  float lneg[128];          // L(sigma) = RN(-log2 sigma) per E4M3 scale code (-inf for 0)
-  double lg2[16];           // log2(i) in double, i = 1..15 (two-level L of sigma * 2^k)
+  float lneg[128];          // fast code rule: L(sigma) = RN(-log2 sigma) per E4M3 scale code (-inf for 0)
 };
 
 // Keep the register results of tcgen05.ld from being read before tcgen05.wait::ld.
@@ -187,11 +186,14 @@ __device__ __forceinline__ UnitGeom unit_geom(int u, const AttnParams& p) {
 //
 // DEC: the decode / split-KV kernels (packed query rows, a split's tile range, partial
 // outputs); the square forward is the DEC = false instance.
-template <int D, int BC, bool SUMP = false, bool DEC = false>
+// FAST: the approximate P_hat code rule (linear-mantissa exponential in the log domain,
+// see phat_pair); the default instances round RN(P * RN(1/sigma)) to E2M1.
+template <int D, int BC, bool SUMP = false, bool DEC = false, bool FAST = false>
 __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     k_attn_fwd(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using C = AttnCfg<D, BC>;
+  static_assert(!(FAST && (SUMP || DEC)), "the fast code rule exists for the plain forward only");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sOnes = smem + C::OFF_ONES;
@@ -246,7 +248,11 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     for (int i = t; i < (int)C::SZ_ONES / 4; i += nt2) reinterpret_cast<uint32_t*>(sOnes)[i] = 0x22222222u;
     for (int i = t; i < 128; i += nt2) reinterpret_cast<uint32_t*>(s1sf)[i] = 0x38383838u;
     fence_proxy_async_smem();
-    for (int i = t; i < 128; i += nt2) rtab[i] = p.lneg[i];
+    if constexpr (FAST) {
+      for (int i = t; i < 128; i += nt2) rtab[i] = p.lneg[i];
+    } else {
+      fill_recip_table(rtab, t, nt2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -609,21 +615,6 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
             alpha_o = __fmul_rn(alpha, __uint_as_float((uint32_t)(127 + k_prev - k2) << 23));
           }
         }
-        float rsum = 0.0f;
-        if constexpr (SUMP) {
-          float part = 0.0f;
-#pragma unroll
-          for (int e = 0; e < CW; e += 2) {
-            const float2 e2 = exp2_own2(__ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2));
-            part = __fadd_rn(__fadd_rn(part, e2.x), e2.y);
-          }
-          float* xs = xsum + (g & 1) * (C::NSW * 128);
-          xs[wg * 128 + row] = part;
-          named_bar(1 + q4, 32 * C::NSW);
-          rsum = xs[row];
-#pragma unroll
-          for (int w2 = 1; w2 < C::NSW; ++w2) rsum = __fadd_rn(rsum, xs[w2 * 128 + row]);
-        }
         // block amax of P = E(fma(block max of S, c, -m_new)), two blocks per packed call
         float pmax[NB];
 #pragma unroll
@@ -634,32 +625,54 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         }
         uint32_t words[CW / 8];
         uint32_t sfw = 0;
+        float part = 0.0f;                   // ablation kernels: this warpgroup's sum of P
 #pragma unroll
         for (int bl = 0; bl < NB; ++bl) {
           float sarg = __fmul_rn(pmax[bl], kSixth);
           if constexpr (SUMP) sarg = __fmul_rn(sarg, kinv);
           const uint32_t sc = cvt_e4m3(sarg);
           sfw |= sc << (8 * bl);
-          float Lb = rtab[sc];
-          if constexpr (SUMP) {
-            if (p.two_level && sc != 0) {
-              // L of the effective scale sigma * 2^k: the integer part lowered by k first
-              const int e4 = (int)(sc >> 3) & 15, m3 = (int)sc & 7;
-              Lb = __double2float_rn(e4 == 0 ? (double)(9 - k2) - p.lg2[m3] : (double)(10 - e4 - k2) - p.lg2[8 + m3]);
+          if constexpr (FAST) {
+            // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
+            const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+              float2 y[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int e = bl * 16 + h8 * 8 + 2 * k;
+                y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
+              }
+              words[2 * bl + h8] = encode8_pairs(y);
+            }
+          } else {
+            // code = E2M1_RN(RN(P * R)), R = RN(1/sigma) (0 for sigma = 0); with the
+            // two-level scale R = RN(1/(sigma 2^k)) = RN(1/sigma) 2^-k, exact
+            float R = rtab[sc];
+            if constexpr (SUMP) R = __fmul_rn(R, kinv);
+            const float2 R2 = make_float2(R, R);
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+              float2 y[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int e = bl * 16 + h8 * 8 + 2 * k;
+                const float2 e2 = exp2_own2(__ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2));
+                if constexpr (SUMP) part = __fadd_rn(__fadd_rn(part, e2.x), e2.y);
+                y[k] = __fmul2_rn(e2, R2);
+              }
+              words[2 * bl + h8] = encode8_pairs(y);
             }
           }
-          // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-          const float B = __fmul_rn(__fadd_rn(__fsub_rn(Lb, mnew), 125.0f), 0.0078125f);
+        }
+        float rsum = 0.0f;
+        if constexpr (SUMP) {
+          float* xs = xsum + (g & 1) * (C::NSW * 128);
+          xs[wg * 128 + row] = part;
+          named_bar(1 + q4, 32 * C::NSW);
+          rsum = xs[row];
 #pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            float2 y[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int e = bl * 16 + h8 * 8 + 2 * k;
-              y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
-            }
-            words[2 * bl + h8] = encode8_pairs(y);
-          }
+          for (int w2 = 1; w2 < C::NSW; ++w2) rsum = __fadd_rn(rsum, xs[w2 * 128 + row]);
         }
         uint8_t* pbuf = sP(pb);
 #pragma unroll
@@ -783,6 +796,7 @@ __global__ void __launch_bounds__(D) k_decode_merge(const DecodeMergeArgs a) {
   }
 }
 
+#ifdef HIFA4_TEST_HOOKS
 // ---------------------------------------------------------------- single-tile probes
 
 // S = Q_hat K_hat^T of one 128 x BC tile through the same TMA / tcgen05.cp / MMA path as
@@ -963,6 +977,71 @@ constexpr uint32_t probe_pv_smem() {
          512 + 64 + 1024;
 }
 
+// P_hat of 16-key blocks by the attention kernel's device steps: block b holds the scores
+// S[16b .. 16b+15] of a row whose running max after the tile is m[b] (an FP16 value).  The
+// block scale comes from E(fma(block max, c, -m)), the codes from the default rule
+// E2M1_RN(RN(E(RN(fma(S, c, -m))) * RN(1/sigma))) or, with FAST, from the fast entry
+// point's linear-mantissa rule.  Writes the E4M3 scale code and 16 E2M1 codes (one per
+// byte) per block.
+struct PhatProbeArgs {
+  const float* S;
+  const float* m;
+  int nblk;
+  float c;
+  float lneg[128];
+  uint8_t* codes;
+  uint8_t* scales;
+};
+
+template <bool FAST>
+__global__ void k_probe_phat(const PhatProbeArgs a) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < a.nblk; b += gridDim.x * blockDim.x) {
+    float s[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) s[e] = a.S[16 * b + e];
+    float bm = s[0];
+#pragma unroll
+    for (int e = 1; e < 15; e += 2) bm = fmax3(bm, s[e], s[e + 1]);
+    bm = fmaxf(bm, s[15]);
+    const float mnew = a.m[b], negm = -mnew;
+    const float c = a.c, c7 = c * 0.0078125f;
+    const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
+    const float pmax = exp2_own2(__ffma2_rn(make_float2(bm, bm), c2, negm2)).x;
+    const uint32_t sc = cvt_e4m3(__fmul_rn(pmax, kSixth));
+    uint32_t words[2];
+    if constexpr (FAST) {
+      const float B = __fmul_rn(__fadd_rn(__fsub_rn(a.lneg[sc], mnew), 125.0f), 0.0078125f);
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float2 y[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = h8 * 8 + 2 * k;
+          y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
+        }
+        words[h8] = encode8_pairs(y);
+      }
+    } else {
+      const float sv = e4m3_value(sc);
+      const float R = (sv > 0.0f && sv <= 448.0f) ? __frcp_rn(sv) : 0.0f;
+      const float2 R2 = make_float2(R, R);
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        float2 y[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = h8 * 8 + 2 * k;
+          y[k] = __fmul2_rn(exp2_own2(__ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2)), R2);
+        }
+        words[h8] = encode8_pairs(y);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 16; ++e) a.codes[16 * b + e] = (uint8_t)((words[e >> 3] >> (4 * (e & 7))) & 0xFu);
+    a.scales[b] = (uint8_t)sc;
+  }
+}
+
 // Elementwise codec check: the device E2M1 / E4M3 conversions and the exp2 on given inputs.
 __global__ void k_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float* ex2) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -972,5 +1051,19 @@ __global__ void k_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m
     ex2[i] = exp2_own(v);
   }
 }
+
+#endif  // HIFA4_TEST_HOOKS
+
+#ifdef HIFA4_TEST_HOOKS
+// The same conversions on the n consecutive fp32 bit patterns start, start + 1, ...
+// (inputs generated on the device, so a whole range needs no input buffer).
+__global__ void k_probe_codec_range(uint32_t start, long long n, uint8_t* e2m1, uint8_t* e4m3) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = __uint_as_float(start + (uint32_t)i);
+    e2m1[i] = (uint8_t)(cvt_e2m1x2(0.0f, v) & 0xF);
+    e4m3[i] = (uint8_t)cvt_e4m3(fabsf(v));
+  }
+}
+#endif  // HIFA4_TEST_HOOKS
 
 }  // namespace hifa4

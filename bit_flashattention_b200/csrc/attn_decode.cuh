@@ -48,7 +48,7 @@ struct DecTCfg {
   static constexpr uint32_t OFF_VSF = OFF_KSF + KS * SZ_KSF;
   static constexpr uint32_t OFF_PSF = OFF_VSF + VS * SZ_VSF;
   static constexpr uint32_t OFF_1SF = OFF_PSF + 2 * SZ_PSF;
-  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;               // 128 x fp32 L(sigma)
+  static constexpr uint32_t OFF_RTAB = OFF_1SF + 512;               // 128 x fp32 RN(1/sigma)
   static constexpr uint32_t OFF_XMAX = OFF_RTAB + 512;              // [2][4 warps][16] fp32 column maxima
   static constexpr uint32_t OFF_BAR = OFF_XMAX + 2 * 4 * 16 * 4;
   // barriers: q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
@@ -176,7 +176,10 @@ __global__ void __launch_bounds__(DecTCfg::NTHREADS, NQ == 16 ? 2 : 3)
     for (int i = t; i < 2 * 1024 / 4; i += 128) reinterpret_cast<uint32_t*>(smem + C::OFF_P)[i] = 0u;
     for (int i = t; i < 2 * (int)C::SZ_PSF / 4; i += 128) reinterpret_cast<uint32_t*>(smem + C::OFF_PSF)[i] = 0u;
     fence_proxy_async_smem();
-    for (int i = t; i < 128; i += 128) rtab[i] = p.lneg[i];
+    for (int i = t; i < 128; i += 128) {   // RN(1/sigma) per E4M3 scale code (0 for sigma = 0)
+      const float sv = e4m3_value((uint32_t)i);
+      rtab[i] = (sv > 0.0f && sv <= 448.0f) ? __frcp_rn(sv) : 0.0f;
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -348,7 +351,6 @@ __global__ void __launch_bounds__(DecTCfg::NTHREADS, NQ == 16 ? 2 : 3)
     const uint32_t lrow = (uint32_t)(q4 * 32) << 16;
     const int b8 = 2 * q4 + (lane >> 4);            // this lane's 16-key block of the tile
     const float c = p.c;
-    const float c7 = c * 0.0078125f;
     const int nv = p.G * p.nq;                      // query rows in use
     // the last key query column q sees: the decode position of its token; unused columns
     // see every key (their Q rows are zero), which keeps their arithmetic finite
@@ -445,10 +447,9 @@ __global__ void __launch_bounds__(DecTCfg::NTHREADS, NQ == 16 ? 2 : 3)
         }
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-          const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc[q]], mnew[q]), 125.0f), 0.0078125f);
-          const float v = __fmaf_rn(fma_sat(s[q], c7, B), 128.0f, kPhatM);
-          y[q] = __uint_as_float(__float_as_uint(v) << 13);
+          // code = E2M1_RN(RN(P * RN(1/sigma))), P = E(RN(fma(S, c, -m_new))); sigma = 0
+          // has R = 0, so every code of that block is 0
+          y[q] = __fmul_rn(exp2_own(__fmaf_rn(s[q], c, -mnew[q])), rtab[sc[q]]);
         }
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {

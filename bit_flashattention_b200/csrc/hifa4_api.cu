@@ -1,5 +1,7 @@
 // Host side of the C ABI declared in include/hifa4.h: argument validation, tensor-map
-// construction, kernel dispatch over the supported (d, kv tile) shapes.
+// construction, kernel dispatch over the supported (d, kv tile) shapes.  Built with
+// HIFA4_TEST_HOOKS defined it also exports the test-only functions of
+// include/hifa4_test.h (the test library; the product library has none of them).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -10,6 +12,9 @@
 #include <vector>
 
 #include "../../include/hifa4.h"
+#ifdef HIFA4_TEST_HOOKS
+#include "../../include/hifa4_test.h"
+#endif
 #include "attn.cuh"
 #include "attn_decode.cuh"
 #include "quant.cuh"
@@ -19,7 +24,6 @@ using namespace hifa4;
 namespace {
 
 unsigned long long g_wait_ns = 2000000000ull;
-int g_inject = 0;
 
 bool device_ok() {
   int dev = 0;
@@ -157,8 +161,8 @@ bool set_smem(K kernel, uint32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
-// L(sigma) = RN_fp32(-log2 sigma) for every non-negative E4M3 scale code, from integer
-// logs in double: normal sigma = (8 + m) 2^(e - 10) gives (10 - e) - log2(8 + m),
+// L(sigma) = RN_fp32(-log2 sigma) for every non-negative E4M3 scale code (the fast P_hat
+// code rule), from integer logs in double: normal sigma = (8 + m) 2^(e - 10) gives (10 - e) - log2(8 + m),
 // subnormal sigma = m 2^-9 gives 9 - log2(m); code 0 (sigma = 0) and the NaN code map to
 // -inf.
 void fill_neg_log2_scales(float* t) {
@@ -173,16 +177,33 @@ void fill_neg_log2_scales(float* t) {
   }
 }
 
+// The streaming quantiser (k_quant_stream) over Q and K row chunks (4096 / d rows each)
+// and V chunks (32 tokens each); the callers set each struct's `units` in those chunks,
+// 0 for a tensor that is not quantised.
+int launch_quant_stream(const QuantRowsArgs& qa, const QuantRowsArgs& ka, const QuantVtArgs& va, int d, int* status,
+                        cudaStream_t stream) {
+  const int units = qa.units + ka.units + va.units;
+  switch (d) {
+    case 64: k_quant_stream<64><<<resident_grid(k_quant_stream<64>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+    case 128: k_quant_stream<128><<<resident_grid(k_quant_stream<128>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+    default: k_quant_stream<256><<<resident_grid(k_quant_stream<256>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
+  }
+  return cuda_status(cudaGetLastError());
+}
+
+int stream_row_chunks(int B, int H, int N, int d) { return B * H * (N / (4096 / d)); }
+
 // Decode / split-KV launch parameters (see AttnParams).
 struct DecodeSpec {
   int nq, G, Nk, nsplit, tps;
   float *part_o, *part_m, *part_l;
 };
 
-template <int D, int BC, bool SUMP = false, bool DEC = false>
+template <int D, int BC, bool SUMP = false, bool DEC = false, bool FAST = false>
 int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                 int N, int causal, void* o, void* m_out, void* l_out, int* status, cudaStream_t stream,
-                int l_from_p = 0, float* trace = nullptr, const DecodeSpec* dec = nullptr, int two_level = 0) {
+                int l_from_p = 0, float* trace = nullptr, const DecodeSpec* dec = nullptr, int two_level = 0,
+                int inject = 0) {
   using C = AttnCfg<D, BC>;
   const int Nk = dec ? dec->Nk : N;
   const uint64_t qrows = dec ? (uint64_t)B * Hkv * 128 : (uint64_t)B * Hq * N;
@@ -194,7 +215,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   // One CTA per SM when it holds all 512 TMEM columns: ask for more than half the SM's
   // shared memory so a second CTA cannot become resident and block in tcgen05.alloc.
   const uint32_t smem = (C::TMEM_COLS == 512 && C::SMEM < 120 * 1024) ? 120 * 1024 : C::SMEM;
-  static bool attr = set_smem(k_attn_fwd<D, BC, SUMP, DEC>, smem);
+  static bool attr = set_smem(k_attn_fwd<D, BC, SUMP, DEC, FAST>, smem);
   if (!attr) return HIFA4_ERR_CUDA;
   AttnParams p;
   std::memset(&p, 0, sizeof(p));
@@ -212,7 +233,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   p.causal = causal ? 1 : 0;
   p.c = (float)(1.4426950408889634074 / std::sqrt((double)D));
   p.wait_ns = g_wait_ns;
-  p.inject = g_inject;
+  p.inject = inject;
   p.l_from_p = l_from_p;
   p.trace = trace;
   p.two_level = two_level;
@@ -228,18 +249,16 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
     p.N = 128;
     p.causal = 0;
   }
-  fill_neg_log2_scales(p.lneg);
-  p.lg2[0] = 0.0;
-  for (int i = 1; i < 16; ++i) p.lg2[i] = std::log2((double)i);
+  if (FAST) fill_neg_log2_scales(p.lneg);
   // persistent grid: as many CTAs as can be resident (TMEM allows 512 / TMEM_COLS per SM);
   // computed once per kernel instance (a function-local static: thread-safe initialisation)
   static const int per_sm = [smem] {
     int n = 0;
-    cudaFuncSetAttribute(k_attn_fwd<D, BC, SUMP, DEC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    cudaFuncSetAttribute(k_attn_fwd<D, BC, SUMP, DEC, FAST>, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_attn_fwd<D, BC, SUMP, DEC, FAST>, C::NTHREADS, smem) != cudaSuccess)
       n = 0;
-    const int m = resident_by_limits(k_attn_fwd<D, BC, SUMP, DEC>, C::NTHREADS, smem);
+    const int m = resident_by_limits(k_attn_fwd<D, BC, SUMP, DEC, FAST>, C::NTHREADS, smem);
     if (m > n) n = m;
     if (n <= 0) n = 1;
     return n < (int)(512 / C::TMEM_COLS) ? n : (int)(512 / C::TMEM_COLS);
@@ -247,7 +266,7 @@ int launch_attn(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qten
   const long long units = dec ? (long long)B * Hkv * dec->nsplit : (long long)B * Hq * (N / 128);
   const long long cap = (long long)per_sm * num_sms();
   const unsigned grid = (unsigned)(units < cap ? units : cap);
-  k_attn_fwd<D, BC, SUMP, DEC><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
+  k_attn_fwd<D, BC, SUMP, DEC, FAST><<<grid, C::NTHREADS, smem, stream>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -315,7 +334,6 @@ int launch_decode_t(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_
   p.part_o = dec.part_o;
   p.part_m = dec.part_m;
   p.part_l = dec.part_l;
-  fill_neg_log2_scales(p.lneg);
   const long long units = (long long)B * Hkv * dec.nsplit;
   const long long cap = (long long)decode_t_resident<NQ>();
   const unsigned grid = (unsigned)(units < cap ? units : cap);
@@ -351,16 +369,16 @@ int attn_validate(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qt
   return HIFA4_OK;
 }
 
-// Validation and dispatch shared by the plain and the ablation entry points.
-template <bool SUMP>
+// Validation and dispatch shared by the plain, fast and ablation entry points.
+template <bool SUMP, bool FAST = false>
 int attn_dispatch(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq, int Hkv,
                   int N, int d, int causal, int kv_tile, void* o, void* m_out, void* l_out, int* status,
-                  cudaStream_t stream, int l_from_p, float* trace, int two_level) {
+                  cudaStream_t stream, int l_from_p, float* trace, int two_level, int inject = 0) {
   const int rc = attn_validate(q, k, vt, B, Hq, Hkv, N, d, kv_tile, o, status);
   if (rc != HIFA4_OK) return rc;
 #define HIFA4_LAUNCH(DD, BB) \
-  launch_attn<DD, BB, SUMP>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, l_from_p, trace, \
-                            nullptr, two_level)
+  launch_attn<DD, BB, SUMP, false, FAST>(q, k, vt, B, Hq, Hkv, N, causal, o, m_out, l_out, status, stream, \
+                                         l_from_p, trace, nullptr, two_level, inject)
   if (d == 64) return kv_tile == 64 ? HIFA4_LAUNCH(64, 64) : HIFA4_LAUNCH(64, 128);
   if (d == 128) {
     if (kv_tile == 256) return HIFA4_LAUNCH(128, 256);
@@ -383,6 +401,7 @@ const char* hifa4_status_string(int s) {
     case HIFA4_ERR_NONFINITE: return "HIFA4_ERR_NONFINITE";
     case HIFA4_ERR_TIMEOUT: return "HIFA4_ERR_TIMEOUT";
     case HIFA4_ERR_CUDA: return "HIFA4_ERR_CUDA";
+    case HIFA4_ERR_IO: return "HIFA4_ERR_IO";
     default: return "HIFA4_ERR_UNKNOWN";
   }
 }
@@ -448,20 +467,14 @@ int hifa4_quantize_qk(const void* q, const void* k, const int64_t q_strides[3], 
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0)) return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
-  const int rows = d == 256 ? 64 : 128;   // rows per unit of k_quant_rows<d>
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
                    nullptr, nullptr, 0, 0,
-                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
+                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), stream_row_chunks(B, Hq, N, d)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
                    nullptr, nullptr, 0, 0,
-                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
-  const int units = qa.units + ka.units;
-  switch (d) {
-    case 64: k_quant_rows<64><<<resident_grid(k_quant_rows<64>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-    case 128: k_quant_rows<128><<<resident_grid(k_quant_rows<128>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-    default: k_quant_rows<256><<<resident_grid(k_quant_rows<256>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-  }
-  return cuda_status(cudaGetLastError());
+                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), stream_row_chunks(B, Hkv, N, d)};
+  QuantVtArgs va{};
+  return launch_quant_stream(qa, ka, va, d, status, stream);
 }
 
 int hifa4_quantize_qk_rope(const void* q, const void* k, const int64_t q_strides[3], const int64_t k_strides[3],
@@ -511,14 +524,10 @@ int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, 
   if (B <= 0 || Hkv <= 0 || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(vt_out, B, Hkv, N, d, 1)) return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
-  QuantVtArgs a{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
-                static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
-  switch (d) {
-    case 64: k_quant_vt<64><<<resident_grid(k_quant_vt<64>, 128, a.units), 128, 0, stream>>>(a, status); break;
-    case 128: k_quant_vt<128><<<resident_grid(k_quant_vt<128>, 128, a.units), 128, 0, stream>>>(a, status); break;
-    default: k_quant_vt<256><<<resident_grid(k_quant_vt<256>, 128, a.units), 128, 0, stream>>>(a, status); break;
-  }
-  return cuda_status(cudaGetLastError());
+  QuantRowsArgs none{};
+  QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
+                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
+  return launch_quant_stream(none, none, va, d, status, stream);
 }
 
 int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_t q_strides[3],
@@ -532,22 +541,15 @@ int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_
   if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0) || !qt_ok(vt_out, B, Hkv, N, d, 1))
     return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
-  const int rows = d == 256 ? 64 : 128;
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
                    nullptr, nullptr, 0, 0,
-                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), B * Hq * (N / rows)};
+                   static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales), stream_row_chunks(B, Hq, N, d)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
                    nullptr, nullptr, 0, 0,
-                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), B * Hkv * (N / rows)};
+                   static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), stream_row_chunks(B, Hkv, N, d)};
   QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
-                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 64)};
-  const int units = qa.units + ka.units + va.units;
-  switch (d) {
-    case 64: k_quant_qkv<64><<<resident_grid(k_quant_qkv<64>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-    case 128: k_quant_qkv<128><<<resident_grid(k_quant_qkv<128>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-    default: k_quant_qkv<256><<<resident_grid(k_quant_qkv<256>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-  }
-  return cuda_status(cudaGetLastError());
+                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
+  return launch_quant_stream(qa, ka, va, d, status, stream);
 }
 
 int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
@@ -555,6 +557,13 @@ int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, con
                              void* l_out, int* status, cudaStream_t stream) {
   return attn_dispatch<false>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream, 0,
                               nullptr, 0);
+}
+
+int hifa4_attn_fwd_quantized_fast(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
+                                  int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
+                                  void* l_out, int* status, cudaStream_t stream) {
+  return attn_dispatch<false, true>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream, 0,
+                                    nullptr, 0);
 }
 
 int hifa4_attn_fwd_ablation(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq,
@@ -707,7 +716,18 @@ int hifa4_read_status(int* status, int clear, cudaStream_t stream) {
 }
 
 void hifa4_set_wait_limit_ns(unsigned long long ns) { g_wait_ns = ns ? ns : 1; }
-void hifa4_debug_set_injection(int mode) { g_inject = mode; }
+
+#ifdef HIFA4_TEST_HOOKS
+// ---------------------------------------------------------------- test-only exports
+// Built only into the test library (libhifa4_test.so, declared in include/hifa4_test.h).
+
+int hifa4_test_attn_fwd_inject(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B, int Hq,
+                               int Hkv, int N, int d, int causal, int kv_tile, int inject, void* o, void* m_out,
+                               void* l_out, int* status, cudaStream_t stream) {
+  if (inject != 0 && inject != 1) return HIFA4_ERR_INVALID_ARG;
+  return attn_dispatch<false>(q, k, vt, B, Hq, Hkv, N, d, causal, kv_tile, o, m_out, l_out, status, stream, 0, nullptr,
+                              0, inject);
+}
 
 int hifa4_probe_qk_tile(const void* q_codes, const void* q_scales, const void* k_codes, const void* k_scales, int d,
                         int kv_tile, float* S, int* status, cudaStream_t stream) {
@@ -763,5 +783,35 @@ int hifa4_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float
   k_probe_codec<<<grid, 256, 0, stream>>>(x, n, e2m1, e4m3, exp2_out);
   return cuda_status(cudaGetLastError());
 }
+
+int hifa4_probe_codec_range(uint32_t start, long long n, uint8_t* e2m1, uint8_t* e4m3, cudaStream_t stream) {
+  if (!e2m1 || !e4m3 || n < 0 || n > (1ll << 32) - (long long)start) return HIFA4_ERR_INVALID_ARG;
+  if (n == 0) return HIFA4_OK;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  k_probe_codec_range<<<num_sms() * 8, 256, 0, stream>>>(start, n, e2m1, e4m3);
+  return cuda_status(cudaGetLastError());
+}
+
+int hifa4_probe_phat(const float* S, const float* m, int nblk, int d, int fast, uint8_t* codes, uint8_t* scales,
+                     cudaStream_t stream) {
+  if (!S || !m || !codes || !scales || nblk < 0 || (fast != 0 && fast != 1)) return HIFA4_ERR_INVALID_ARG;
+  if (!d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
+  if (nblk == 0) return HIFA4_OK;
+  if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  PhatProbeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.S = S;
+  a.m = m;
+  a.nblk = nblk;
+  a.c = (float)(1.4426950408889634074 / std::sqrt((double)d));
+  fill_neg_log2_scales(a.lneg);
+  a.codes = codes;
+  a.scales = scales;
+  const int grid = (nblk + 127) / 128 < 1024 ? (nblk + 127) / 128 : 1024;
+  if (fast) k_probe_phat<true><<<grid, 128, 0, stream>>>(a);
+  else k_probe_phat<false><<<grid, 128, 0, stream>>>(a);
+  return cuda_status(cudaGetLastError());
+}
+#endif  // HIFA4_TEST_HOOKS
 
 }  // extern "C"

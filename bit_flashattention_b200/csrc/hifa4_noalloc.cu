@@ -12,7 +12,10 @@
 // life of the process.  All calls on a device share it and it keeps whatever the last
 // call wrote: calls whose GPU work overlaps (different streams, no ordering between them)
 // race on it.  Nothing in it needs to start at zero -- every call rewrites all the bytes
-// it reads (V^T codes and scale atoms, padding rows included).
+// it reads (V^T codes and scale atoms, padding rows included).  The array's device
+// address is looked up once per device and cached; a cudaDeviceReset (or any other
+// teardown of the device's primary context) invalidates it, so this entry point must not
+// be used again in a process after such a reset.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -30,14 +33,29 @@ void* g_scratch_ptr[64] = {};
 
 // Device address of g_vt_scratch on the current device.  In host code the symbol is only
 // a host-side stand-in, so the address is looked up once per device (with that device
-// current) and cached.
+// current) and cached.  A device that is not sm_100 is reported as such before any
+// lookup (this library holds no code for it); a failed lookup clears the runtime's
+// sticky last-error so that it does not surface in a later, unrelated call.
 int scratch_address(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HIFA4_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return HIFA4_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (major != 10 || minor != 0) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   std::lock_guard<std::mutex> lk(g_mu);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_vt_scratch) != cudaSuccess || p == nullptr) return HIFA4_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_vt_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return HIFA4_ERR_CUDA;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];

@@ -15,14 +15,14 @@ namespace hifa4 {
 // RN(1/6) in fp32.
 constexpr float kSixth = 0x1.555556p-3f;
 
-// The softmax's exp2: E(x) = p(f) * 2^n with x' = max(x, -127), n = floor(x'), f = x' - n
-// and p(f) = (c2 f + c1) f + 1 evaluated with fused multiply-adds; the coefficients are a
-// minimax fit of 2^f on [0, 1) in relative error with p(0) = 1 held exact (max relative
-// error 2.05e-3, far below the spacing of the 4-bit codes P is rounded to).  The floor
-// uses a round-down add of 1.5 * 2^23, whose low mantissa bits then hold n, so the
-// exponent insert is one integer multiply-add.
-constexpr float kExp2C1 = 0x1.54f8d6p-1f;
-constexpr float kExp2C2 = 0x1.51d9ccp-2f;
+// The softmax's exp2: E(x) = p(f) * 2^n with x' = max(x, -127), n = floor(x'),
+// f = RN(x' - n) and p(f) = ((c3 f + c2) f + c1) f + 1 evaluated with fused multiply-adds;
+// the coefficients are a minimax fit of 2^f on [0, 1) in relative error with p(0) = 1 held
+// exact (max relative error 8.6e-5).  The floor uses a round-down add of 1.5 * 2^23, whose
+// low mantissa bits then hold n, so the exponent insert is one integer multiply-add.
+constexpr float kExp2C1 = 0x1.63e65ap-1f;
+constexpr float kExp2C2 = 0x1.d23788p-3f;
+constexpr float kExp2C3 = 0x1.3baaa8p-4f;
 
 // bits(p) + (n << 23), with n in the low bits of v's pattern (v = floor(x') + 1.5 * 2^23).
 __device__ __forceinline__ float insert_exponent(float p, float v) {
@@ -35,8 +35,8 @@ __device__ __forceinline__ float exp2_own(float x) {
   const float xc = fmaxf(x, -127.0f);
   const float v = __fadd_rd(xc, 12582912.0f);
   const float n = __fsub_rn(v, 12582912.0f);
-  const float f = __fsub_rn(xc, n);
-  const float p = __fmaf_rn(__fmaf_rn(kExp2C2, f, kExp2C1), f, 1.0f);
+  const float f = __fsub_rn(xc, n);                                        // RN(xc - n)
+  const float p = __fmaf_rn(__fmaf_rn(__fmaf_rn(kExp2C3, f, kExp2C2), f, kExp2C1), f, 1.0f);
   return insert_exponent(p, v);
 }
 
@@ -46,21 +46,25 @@ __device__ __forceinline__ float2 exp2_own2(float2 x) {
   const float2 xc = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
   const float2 v = __fadd2_rd(xc, make_float2(12582912.0f, 12582912.0f));
   const float2 n = __fadd2_rn(v, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);          // xc - n, exact
-  float2 p = __ffma2_rn(make_float2(kExp2C2, kExp2C2), f, make_float2(kExp2C1, kExp2C1));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);          // RN(xc - n)
+  float2 p = __ffma2_rn(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
   p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
   return make_float2(insert_exponent(p.x, v.x), insert_exponent(p.y, v.y));
 }
 
-// P_hat code decision in the log domain.  With the per-block bias
+// P_hat codes, fast approximate form (a separate entry point, never the default): the
+// code of a score is decided in the log domain.  With the per-block bias
 // B = (L(sigma) - m + 125)/128, L(sigma) = RN(-log2 sigma), a score's u = sat(S * c/128 + B)
 // holds log2(P / sigma) + 125 scaled into [0, 1].  The code is the E2M1 rounding of the
 // linear-mantissa exponential y = 2^floor(z) * (1 + frac z) of z = 128 u - 125 + delta on a
-// 2^-10 grid (delta = -73/1024 centres the E2M1 rounding boundaries on those of the exact
-// exponential).  One fma forms v = 128 u + kPhatM, kPhatM = 8194 + delta: v lies in
-// [2^13, 2^14), whose spacing is 2^-10, so v's mantissa field is (z + 127) * 2^10, and
-// shifting v's bits left by 13 leaves exactly the bits of y (exponent floor(z) + 127, top
-// ten mantissa bits frac z).
+// 2^-10 grid (delta = -73/1024 puts the E2M1 rounding boundaries within 0.014 log2 units
+// of those of the exact exponential, the lowest within 0.071).  One fma forms
+// v = 128 u + kPhatM, kPhatM = 8194 + delta: v lies in [2^13, 2^14), whose spacing is
+// 2^-10, so v's mantissa field is (z + 127) * 2^10, and shifting v's bits left by 13
+// leaves exactly the bits of y (exponent floor(z) + 127, top ten mantissa bits frac z).
+// The default path instead rounds RN(P * RN(1/sigma)) to E2M1, the block quantiser's
+// own rule.
 constexpr float kPhatM = 8193.9287109375f;   // 8194 - 73/1024
 
 __device__ __forceinline__ float fma_sat(float a, float b, float c) {

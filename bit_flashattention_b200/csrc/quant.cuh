@@ -209,20 +209,6 @@ __device__ __forceinline__ void quant_rows_rope_pair(const QuantRowsArgs& a, int
   bad |= !isfinite(nan_acc);
 }
 
-// Grid-stride over Q units then K units.
-template <int D>
-__global__ void __launch_bounds__(256) k_quant_rows(QuantRowsArgs qa, QuantRowsArgs ka, int* status) {
-  __shared__ float rtab[256];
-  fill_recip_table(rtab, threadIdx.x, 256);
-  __syncthreads();
-  bool bad = false;
-  for (int u = blockIdx.x; u < qa.units + ka.units; u += gridDim.x) {
-    if (u < qa.units) quant_rows_unit<D>(qa, u, rtab, bad);
-    else quant_rows_unit<D>(ka, u - qa.units, rtab, bad);
-  }
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
-}
-
 // Decode Q packing + Smooth-QK + quantise: one 128-row unit per (batch, kv head).
 template <int D>
 __global__ void __launch_bounds__(256) k_quant_q_decode(QuantRowsArgs qa, int* status) {
@@ -258,39 +244,98 @@ struct QuantVtArgs {
   int units;                  // B * Hkv * N / TOK for the kernel's TOK
 };
 
-// One unit (TOK consecutive tokens of one kv head, TOK = 32 with 128 threads or 64 with
-// 256 threads) of the transposing V quantiser.  The TOK x D tile is staged in shared
-// memory with coalesced 16-byte loads (all of a thread's loads in flight first); then item
-// (channel c, 32-token half) quantises the half's two 16-token blocks of channel c and
-// writes their 16 code bytes and its 2 bytes of the channel's scale word.  For D = 64 the
-// unused rows 64..127 of the 128-channel atom are zeroed.
-template <int D, int TOK, int NT>
-__device__ __forceinline__ void quant_vt_unit(const QuantVtArgs& a, int unit, __nv_bfloat16* tile, const float* rtab,
-                                              bool& bad) {
-  constexpr int NAV = (D + 127) / 128;
-  constexpr int LD = D + 8;                     // padded staging row (bf16 elements)
-  constexpr int LOADS = TOK * (D / 8) / NT;     // 16-byte loads per thread
-  const int nunit = a.N / TOK;
-  const int bh = unit / nunit, t0 = (unit % nunit) * TOK;
-  const int b = bh / a.H, h = bh % a.H;
-  const __nv_bfloat16* src = a.v + b * a.sb + h * a.sh + (long long)t0 * a.sn;
-  uint4 raw[LOADS];
+// ---------------------------------------------------------------- streaming quantiser
+// Q, K (rows, blocks along d) and V^T (blocks along tokens) as one stream of 8 KB chunks:
+// a row chunk is 4096 / D rows of one head (thread t: row t / (D/16), 16-element block
+// t % (D/16), two 16-byte loads), a V chunk is 32 tokens of one kv head (D/64 16-byte loads
+// per thread, staged through shared memory for the transpose).  Chunk c goes to CTA
+// c % gridDim.x, Q chunks first, then K, then V, so every CTA gets the same number of
+// chunks to within one.  Each thread keeps the loads of its next two chunks in flight
+// while it quantises the current one (registers, three buffers by static index).
+template <int D>
+struct StreamCfg {
+  static constexpr int NT = 256;
+  static constexpr int RC = 4096 / D;                 // rows per row chunk
+  static constexpr int LV = D / 64;                   // 16-byte loads per thread of a V chunk
+  static constexpr int NL = LV > 2 ? LV : 2;          // loads per thread of any chunk
+  static constexpr int LD = D + 8;                    // padded V staging row (bf16)
+};
+
+template <int D>
+struct StreamChunk {
+  int kind;                                           // 0 Q, 1 K, 2 V, -1 none
+  int idx;                                            // chunk index within its tensor
+};
+
+template <int D>
+__device__ __forceinline__ StreamChunk<D> stream_chunk(int c, const QuantRowsArgs& qa, const QuantRowsArgs& ka,
+                                                       const QuantVtArgs& va) {
+  if (c < qa.units) return {0, c};
+  c -= qa.units;
+  if (c < ka.units) return {1, c};
+  c -= ka.units;
+  if (c < va.units) return {2, c};
+  return {-1, 0};
+}
+
+template <int D>
+__device__ __forceinline__ void stream_load(const StreamChunk<D>& ch, const QuantRowsArgs& qa, const QuantRowsArgs& ka,
+                                            const QuantVtArgs& va, uint4 (&r)[StreamCfg<D>::NL]) {
+  using C = StreamCfg<D>;
+  if (ch.kind == 0 || ch.kind == 1) {
+    const QuantRowsArgs& a = ch.kind == 0 ? qa : ka;
+    const int per_head = a.N / C::RC;
+    const int bh = ch.idx / per_head, row = (ch.idx % per_head) * C::RC + threadIdx.x / (D / 16);
+    const int b = bh / a.H, h = bh % a.H;
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + b * a.sb + h * a.sh + (long long)row * a.sn +
+                                                      (threadIdx.x % (D / 16)) * 16);
+    r[0] = src[0];
+    r[1] = src[1];
+  } else if (ch.kind == 2) {
+    const int per_head = va.N / 32;
+    const int bh = ch.idx / per_head, t0 = (ch.idx % per_head) * 32;
+    const int b = bh / va.H, h = bh % va.H;
+    const __nv_bfloat16* src = va.v + b * va.sb + h * va.sh + (long long)t0 * va.sn;
 #pragma unroll
-  for (int k = 0; k < LOADS; ++k) {
-    const int it = threadIdx.x + k * NT;
-    raw[k] = *reinterpret_cast<const uint4*>(src + (it / (D / 8)) * a.sn + (it % (D / 8)) * 8);
+    for (int k = 0; k < C::LV; ++k) {
+      const int it = threadIdx.x + k * C::NT;
+      r[k] = *reinterpret_cast<const uint4*>(src + (it / (D / 8)) * va.sn + (it % (D / 8)) * 8);
+    }
   }
-  __syncthreads();                            // the previous unit's readers are done with the tile
+}
+
+template <int D>
+__device__ __forceinline__ void stream_rows(const QuantRowsArgs& a, int idx, const uint4 (&r)[StreamCfg<D>::NL],
+                                            const float* rtab, float& nan_acc) {
+  using C = StreamCfg<D>;
+  const int per_head = a.N / C::RC;
+  const int bh = idx / per_head, row = (idx % per_head) * C::RC + threadIdx.x / (D / 16);
+  const int g = (bh % a.H) / (a.H / a.Hkv);
+  const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&r[0]);
+  float2 v[8];
 #pragma unroll
-  for (int k = 0; k < LOADS; ++k) {
-    const int it = threadIdx.x + k * NT;
-    *reinterpret_cast<uint4*>(&tile[(it / (D / 8)) * LD + (it % (D / 8)) * 8]) = raw[k];
+  for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
+  quant_block16<D>(a, bh, g, row, threadIdx.x % (D / 16), v, rtab, nan_acc);
+}
+
+// V chunk: 32 tokens x D channels staged in `tile`; item c (channel) quantises the chunk's
+// two 16-token blocks of channel c: 16 code bytes and 2 bytes of the channel's scale word.
+template <int D>
+__device__ __forceinline__ void stream_vt(const QuantVtArgs& a, int idx, const uint4 (&r)[StreamCfg<D>::NL],
+                                          __nv_bfloat16* tile, const float* rtab, float& nan_acc) {
+  using C = StreamCfg<D>;
+  constexpr int NAV = (D + 127) / 128;
+  const int per_head = a.N / 32;
+  const int bh = idx / per_head, half = idx % per_head, ch = half >> 1, hb = half & 1;
+  __syncthreads();                                    // the previous V chunk's readers are done
+#pragma unroll
+  for (int k = 0; k < C::LV; ++k) {
+    const int it = threadIdx.x + k * C::NT;
+    *reinterpret_cast<uint4*>(&tile[(it / (D / 8)) * C::LD + (it % (D / 8)) * 8]) = r[k];
   }
   __syncthreads();
-#pragma unroll
-  for (int it = threadIdx.x; it < (TOK / 32) * D; it += NT) {
-    const int c = it % D, hh = it / D;
-    const int half = t0 / 32 + hh, ch = half >> 1, hb = half & 1;
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
     uint32_t w[4];
     uint32_t sc2 = 0;
 #pragma unroll
@@ -299,11 +344,11 @@ __device__ __forceinline__ void quant_vt_unit(const QuantVtArgs& a, int unit, __
       float amax = 0.0f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        x[e] = make_float2(__bfloat162float(tile[(hh * 32 + blk * 16 + 2 * e) * LD + c]),
-                           __bfloat162float(tile[(hh * 32 + blk * 16 + 2 * e + 1) * LD + c]));
+        x[e] = make_float2(__bfloat162float(tile[(blk * 16 + 2 * e) * C::LD + c]),
+                           __bfloat162float(tile[(blk * 16 + 2 * e + 1) * C::LD + c]));
         amax = max3_abs_nan(amax, x[e].x, x[e].y);
       }
-      bad |= !isfinite(amax);
+      nan_acc = max3_abs_nan(nan_acc, amax, amax);
       float R;
       sc2 |= block_scale_tab(amax, rtab, R) << (8 * blk);
       const float2 R2 = make_float2(R, R);
@@ -320,42 +365,56 @@ __device__ __forceinline__ void quant_vt_unit(const QuantVtArgs& a, int unit, __
         make_uint4(w[0], w[1], w[2], w[3]);
     uint8_t* atom = a.sf + (((long long)bh * (a.N / 64) + ch) * NAV + c / 128) * 512;
     *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(c % 128, 2 * hb)) = (uint16_t)sc2;
-  }
-  if constexpr (D < 128) {
-    constexpr int PAD = 128 - D;
-    for (int it = threadIdx.x; it < (TOK / 32) * PAD; it += NT) {
-      const int half = t0 / 32 + it / PAD, r = D + it % PAD;
-      uint8_t* atom = a.sf + ((long long)bh * (a.N / 64) + (half >> 1)) * NAV * 512;
-      *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(r, 2 * (half & 1))) = 0;
-    }
+  } else if (D < 128 && threadIdx.x < 128) {
+    // rows D..127 of the 128-channel atom are zero (D = 64)
+    uint8_t* atom = a.sf + ((long long)bh * (a.N / 64) + ch) * NAV * 512;
+    *reinterpret_cast<uint16_t*>(atom + sf_atom_offset(threadIdx.x, 2 * hb)) = 0;
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) k_quant_vt(QuantVtArgs a, int* status) {
-  __shared__ __align__(16) __nv_bfloat16 tile[32 * (D + 8)];
-  __shared__ float rtab[256];
-  fill_recip_table(rtab, threadIdx.x, 128);
-  bool bad = false;
-  for (int u = blockIdx.x; u < a.units; u += gridDim.x) quant_vt_unit<D, 32, 128>(a, u, tile, rtab, bad);
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+__device__ __forceinline__ void stream_compute(const StreamChunk<D>& ch, const QuantRowsArgs& qa,
+                                               const QuantRowsArgs& ka, const QuantVtArgs& va,
+                                               const uint4 (&r)[StreamCfg<D>::NL], __nv_bfloat16* tile,
+                                               const float* rtab, float& nan_acc) {
+  if (ch.kind == 0) stream_rows<D>(qa, ch.idx, r, rtab, nan_acc);
+  else if (ch.kind == 1) stream_rows<D>(ka, ch.idx, r, rtab, nan_acc);
+  else if (ch.kind == 2) stream_vt<D>(va, ch.idx, r, tile, rtab, nan_acc);
 }
 
-// Q, K and V in one launch: grid-stride over Q and K row units, then 64-token V units.
+// Q and K row chunks (qa.units, ka.units: rows / (4096 / D)) and V chunks (va.units:
+// tokens / 32), any of the three counts may be 0.
 template <int D>
-__global__ void __launch_bounds__(256) k_quant_qkv(QuantRowsArgs qa, QuantRowsArgs ka, QuantVtArgs va, int* status) {
-  __shared__ __align__(16) __nv_bfloat16 tile[64 * (D + 8)];
+__global__ void __launch_bounds__(256, D == 256 ? 2 : 4) k_quant_stream(QuantRowsArgs qa, QuantRowsArgs ka, QuantVtArgs va,
+                                                         int* status) {
+  using C = StreamCfg<D>;
+  __shared__ __align__(16) __nv_bfloat16 tile[32 * C::LD];
   __shared__ float rtab[256];
   fill_recip_table(rtab, threadIdx.x, 256);
   __syncthreads();
-  bool bad = false;
-  const int nrows = qa.units + ka.units;
-  for (int u = blockIdx.x; u < nrows + va.units; u += gridDim.x) {
-    if (u < qa.units) quant_rows_unit<D>(qa, u, rtab, bad);
-    else if (u < nrows) quant_rows_unit<D>(ka, u - qa.units, rtab, bad);
-    else quant_vt_unit<D, 64, 256>(va, u - nrows, tile, rtab, bad);
+  const int total = qa.units + ka.units + va.units;
+  const int G = gridDim.x;
+  float nan_acc = 0.0f;
+  uint4 b0[C::NL], b1[C::NL], b2[C::NL];
+  int c = blockIdx.x;
+  StreamChunk<D> k0 = stream_chunk<D>(c, qa, ka, va), k1 = stream_chunk<D>(c + G, qa, ka, va), k2;
+  stream_load<D>(k0, qa, ka, va, b0);
+  stream_load<D>(k1, qa, ka, va, b1);
+  // the chunk kind is uniform over the CTA, so the __syncthreads of V chunks are reached by all
+  for (; c < total; c += 3 * G) {
+    k2 = stream_chunk<D>(c + 2 * G, qa, ka, va);
+    stream_load<D>(k2, qa, ka, va, b2);
+    stream_compute<D>(k0, qa, ka, va, b0, tile, rtab, nan_acc);
+    if (c + G >= total) break;
+    k0 = stream_chunk<D>(c + 3 * G, qa, ka, va);
+    stream_load<D>(k0, qa, ka, va, b0);
+    stream_compute<D>(k1, qa, ka, va, b1, tile, rtab, nan_acc);
+    if (c + 2 * G >= total) break;
+    k1 = stream_chunk<D>(c + 4 * G, qa, ka, va);
+    stream_load<D>(k1, qa, ka, va, b1);
+    stream_compute<D>(k2, qa, ka, va, b2, tile, rtab, nan_acc);
   }
-  if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
+  if (__any_sync(0xffffffffu, !isfinite(nan_acc)) && (threadIdx.x & 31) == 0) atomicOr(status, ST_NONFINITE);
 }
 
 struct AmaxArgs {

@@ -86,19 +86,23 @@ def head_slab(w: Workload, which: str, b: int, h: int, calib: bool = False) -> n
     return f32_to_bf16_bits(x)
 
 
-def tensor(w: Workload, which: str, calib: bool = False) -> np.ndarray:
-    """Full [B, H, N, d] bf16 tensor (uint16 bits) for 'q', 'k' or 'v'."""
+def tensor(w: Workload, which: str, calib: bool = False, batches=None) -> np.ndarray:
+    """[B, H, N, d] bf16 tensor (uint16 bits) for 'q', 'k' or 'v'; with `batches` (a range of
+    batch indices) only those batches, [len(batches), H, N, d], drawn exactly as in the
+    full tensor."""
     H = w.Hq if which == "q" else w.Hkv
-    out = np.empty((w.B, H, w.N, w.d), dtype=np.uint16)
-    for b in range(w.B):
+    bs = range(w.B) if batches is None else batches
+    out = np.empty((len(bs), H, w.N, w.d), dtype=np.uint16)
+    for i, b in enumerate(bs):
         for h in range(H):
-            out[b, h] = head_slab(w, which, b, h, calib)
+            out[i, h] = head_slab(w, which, b, h, calib)
     return out
 
 
-def inputs(w: Workload, calib: bool = False):
-    """(Q, K, V) bf16 bit tensors of the workload (or of its calibration sample)."""
-    return tensor(w, "q", calib), tensor(w, "k", calib), tensor(w, "v", calib)
+def inputs(w: Workload, calib: bool = False, batches=None):
+    """(Q, K, V) bf16 bit tensors of the workload (or of its calibration sample); `batches`
+    selects a range of batch indices."""
+    return tensor(w, "q", calib, batches), tensor(w, "k", calib, batches), tensor(w, "v", calib, batches)
 
 
 def sample_rows(w: Workload, per_head: int = 8, seed: int = 7, br: int = 128):

@@ -15,7 +15,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libhifa4.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "hifa4.h")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_NONFINITE, ERR_TIMEOUT, ERR_CUDA = range(7)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_UNSUPPORTED_DEVICE, ERR_NONFINITE, ERR_TIMEOUT, ERR_CUDA, ERR_IO = range(8)
 
 
 class Hifa4Error(RuntimeError):
@@ -53,6 +53,7 @@ def lib():
             "hifa4_rope_table": ([ctypes.c_double, i, i, i, P, P], i),
             "hifa4_quantize_qkv": ([P, P, P, P, P, P, i, i, i, i, i, P, P, QP, QP, QP, P, P], i),
             "hifa4_attn_fwd_quantized": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
+            "hifa4_attn_fwd_quantized_fast": ([QP, QP, QP, i, i, i, i, i, i, i, P, P, P, P, P], i),
             "hifa4_attn_fwd_ablation": ([QP, QP, QP, i, i, i, i, i, i, i, i, i, P, P, P, P, P, P], i),
             "hifa4_quantize_q_decode": ([P, P, i, i, i, i, i, P, QP, P, P], i),
             "hifa4_decode_workspace_bytes": ([i, i, i, i], sz),
@@ -61,10 +62,8 @@ def lib():
             "hifa4_attn_fwd": ([QP, QP, P, P, i, i, i, i, i, i, i, P, sz, P, P, P, P, P], i),
             "hifa4_read_status": ([P, i, P], i),
             "hifa4_set_wait_limit_ns": ([ull], None),
-            "hifa4_debug_set_injection": ([i], None),
-            "hifa4_probe_qk_tile": ([P, P, P, P, i, i, P, P, P], i),
-            "hifa4_probe_pv_tile": ([P, P, P, P, i, i, P, P, P, P], i),
-            "hifa4_probe_codec": ([P, i, P, P, P, P], i),
+            "hifa4_calibration_save": ([ctypes.c_char_p, i, i, f, P, P], i),
+            "hifa4_calibration_load": ([ctypes.c_char_p, P, P, P, P, P, sz], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -74,9 +73,9 @@ def lib():
     return _lib
 
 
-def declared_functions():
-    """Names of the functions include/hifa4.h declares."""
-    txt = open(HEADER_PATH).read()
+def declared_functions(header=HEADER_PATH):
+    """Names of the functions a header of this library (default include/hifa4.h) declares."""
+    txt = open(header).read()
     return sorted(set(re.findall(r"HIFA4_API\s+[\w\s\*]+?\b(hifa4_\w+)\s*\(", txt)))
 
 
@@ -175,10 +174,6 @@ def hifa4_set_wait_limit_ns(ns: int):
     lib().hifa4_set_wait_limit_ns(int(ns))
 
 
-def hifa4_debug_set_injection(mode: int):
-    lib().hifa4_debug_set_injection(int(mode))
-
-
 def hifa4_calibrate_smooth(q_cal, k_cal, alpha: float):
     """Smooth-QK scales (s, s_inv), fp32 [Hkv, d] on q_cal's device.  Synchronises."""
     _need(q_cal, torch.bfloat16, "q_cal")
@@ -192,6 +187,32 @@ def hifa4_calibrate_smooth(q_cal, k_cal, alpha: float):
     _check(lib().hifa4_calibrate_smooth(_ptr(q_cal), _ptr(k_cal), _strides(q_cal), _strides(k_cal), B, Hq, Hkv, N, d,
                                         float(alpha), _ptr(s), _ptr(si), _ptr(ws), _stream()), "hifa4_calibrate_smooth")
     return s, si
+
+
+def hifa4_calibration_save(path, s, sinv, alpha: float):
+    """Write the Smooth-QK scales s, s_inv (fp32 [Hkv, d], any device) and alpha to `path`."""
+    import numpy as np
+    sh = np.ascontiguousarray(s.detach().float().cpu().numpy())
+    sih = np.ascontiguousarray(sinv.detach().float().cpu().numpy())
+    if sh.ndim != 2 or sih.shape != sh.shape:
+        raise ValueError("s and sinv must both be [Hkv, d]")
+    _check(lib().hifa4_calibration_save(os.fsencode(path), sh.shape[0], sh.shape[1], float(alpha),
+                                        sh.ctypes.data_as(ctypes.c_void_p), sih.ctypes.data_as(ctypes.c_void_p)),
+           "hifa4_calibration_save")
+
+
+def hifa4_calibration_load(path, device=None):
+    """Read a calibration file -> (s, s_inv fp32 [Hkv, d] on `device`, alpha)."""
+    import numpy as np
+    hk, dd, al = ctypes.c_int(), ctypes.c_int(), ctypes.c_float()
+    _check(lib().hifa4_calibration_load(os.fsencode(path), ctypes.byref(hk), ctypes.byref(dd), ctypes.byref(al), None,
+                                        None, 0), "hifa4_calibration_load")
+    sh = np.empty((hk.value, dd.value), np.float32)
+    sih = np.empty_like(sh)
+    _check(lib().hifa4_calibration_load(os.fsencode(path), ctypes.byref(hk), ctypes.byref(dd), ctypes.byref(al),
+                                        sh.ctypes.data_as(ctypes.c_void_p), sih.ctypes.data_as(ctypes.c_void_p),
+                                        sh.size), "hifa4_calibration_load")
+    return torch.from_numpy(sh).to(device), torch.from_numpy(sih).to(device), float(al.value)
 
 
 def hifa4_quantize_qk(q, k, s=None, sinv=None, status=None, out=None):
@@ -280,16 +301,18 @@ def _outputs(B, Hq, N, d, dev, o, m, l):
     return o, m, l
 
 
-def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=None, m=None, l=None):
-    """The fused 4-bit attention of already quantised Q, K and V^T -> (O bf16, m fp16, l fp16)."""
+def hifa4_attn_fwd_quantized(qq, kq, vt, causal=True, kv_tile=0, status=None, o=None, m=None, l=None,
+                             fast=False):
+    """The fused 4-bit attention of already quantised Q, K and V^T -> (O bf16, m fp16, l fp16).
+    fast=True calls hifa4_attn_fwd_quantized_fast (the approximate P_hat code rule)."""
     for t, w in ((qq, "q"), (kq, "k"), (vt, "vt")):
         _need_qt(t, w)
     dev = qq.codes.device
     o, m, l = _outputs(qq.B, qq.H, qq.N, qq.d, dev, o, m, l)
     st = _status(status, dev)
-    _check(lib().hifa4_attn_fwd_quantized(qq.c(), kq.c(), vt.c(), qq.B, qq.H, kq.H, qq.N, qq.d, int(causal),
-                                          int(kv_tile), _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()),
-           "hifa4_attn_fwd_quantized")
+    name = "hifa4_attn_fwd_quantized_fast" if fast else "hifa4_attn_fwd_quantized"
+    _check(getattr(lib(), name)(qq.c(), kq.c(), vt.c(), qq.B, qq.H, kq.H, qq.N, qq.d, int(causal), int(kv_tile),
+                                _ptr(o), _ptr(m), _ptr(l), _ptr(st), _stream()), name)
     return o, m, l
 
 
@@ -371,34 +394,3 @@ def hifa4_attn_fwd(qq, kq, v, causal=True, kv_tile=0, status=None, workspace=Non
 
 def hifa4_attn_workspace_bytes(B, Hkv, N, d):
     return lib().hifa4_attn_workspace_bytes(B, Hkv, N, d)
-
-
-def hifa4_probe_qk_tile(q_codes, q_scales, k_codes, k_scales, d, kv_tile, status=None):
-    for t, w in ((q_codes, "q_codes"), (q_scales, "q_scales"), (k_codes, "k_codes"), (k_scales, "k_scales")):
-        _need(t, torch.uint8, w, contiguous=True)
-    S = torch.empty(128, kv_tile, dtype=torch.float32, device=q_codes.device)
-    st = _status(status, q_codes.device)
-    _check(lib().hifa4_probe_qk_tile(_ptr(q_codes), _ptr(q_scales), _ptr(k_codes), _ptr(k_scales), d, kv_tile, _ptr(S),
-                                     _ptr(st), _stream()), "hifa4_probe_qk_tile")
-    return S
-
-
-def hifa4_probe_pv_tile(p_codes, p_scales, vt_codes, vt_scales, d, kv_tile, status=None):
-    for t, w in ((p_codes, "p_codes"), (p_scales, "p_scales"), (vt_codes, "vt_codes"), (vt_scales, "vt_scales")):
-        _need(t, torch.uint8, w, contiguous=True)
-    O = torch.empty(128, d, dtype=torch.float32, device=p_codes.device)
-    R = torch.empty(128, dtype=torch.float32, device=p_codes.device)
-    st = _status(status, p_codes.device)
-    _check(lib().hifa4_probe_pv_tile(_ptr(p_codes), _ptr(p_scales), _ptr(vt_codes), _ptr(vt_scales), d, kv_tile, _ptr(O),
-                                     _ptr(R), _ptr(st), _stream()), "hifa4_probe_pv_tile")
-    return O, R
-
-
-def hifa4_probe_codec(x):
-    _need(x, torch.float32, "x", contiguous=True)
-    n = x.numel()
-    e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
-    e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
-    ex = torch.empty(n, dtype=torch.float32, device=x.device)
-    _check(lib().hifa4_probe_codec(_ptr(x), n, _ptr(e2), _ptr(e4), _ptr(ex), _stream()), "hifa4_probe_codec")
-    return e2, e4, ex

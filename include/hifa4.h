@@ -62,7 +62,8 @@ typedef enum {
   HIFA4_ERR_UNSUPPORTED_DEVICE = 3,/* current device is not sm_100 */
   HIFA4_ERR_NONFINITE = 4,         /* a quantised input held inf or NaN (device-detected) */
   HIFA4_ERR_TIMEOUT = 5,           /* a kernel's bounded wait ran out (device-detected) */
-  HIFA4_ERR_CUDA = 6               /* a CUDA runtime call or launch failed */
+  HIFA4_ERR_CUDA = 6,              /* a CUDA runtime call or launch failed */
+  HIFA4_ERR_IO = 7                 /* a calibration file could not be written or read, or is not valid */
 } hifa4_status;
 
 /* Device status-word bits (ORed by kernels into the caller's `int* status`). */
@@ -114,6 +115,25 @@ HIFA4_API size_t hifa4_calibrate_workspace_bytes(int Hkv, int d);
 HIFA4_API int hifa4_calibrate_smooth(const void* q_cal, const void* k_cal, const int64_t q_strides[3],
                            const int64_t k_strides[3], int B, int Hq, int Hkv, int N, int d, float alpha,
                            float* s_out, float* sinv_out, void* workspace, cudaStream_t stream);
+
+/*
+ * The Smooth-QK calibration as a file: the method's one persistent artefact (the HiFA4
+ * abstract fixes the scales offline, so they are computed once and shipped with the
+ * model).  HOST arrays; copy them to or from the device yourself.  Layout (little-endian):
+ * magic "HIFA4CAL", uint32 version = 1, int32 Hkv, int32 d, fp32 alpha, uint32 CRC-32 of
+ * the arrays, then s [Hkv * d] and s_inv [Hkv * d] fp32, exactly as
+ * hifa4_calibrate_smooth produced them (bit patterns are preserved).
+ *   hifa4_calibration_save: HIFA4_ERR_INVALID_ARG for null arrays or path, Hkv or d not
+ *     positive, alpha negative or NaN; HIFA4_ERR_IO if the file cannot be written.
+ *   hifa4_calibration_load: reads the header into *Hkv, *d, *alpha; with s and sinv both
+ *     NULL it stops there (to size the arrays), otherwise it needs capacity >= Hkv * d
+ *     (else HIFA4_ERR_INVALID_ARG) and fills both.  HIFA4_ERR_IO for a missing or short
+ *     file, a wrong magic or version, trailing bytes or a CRC mismatch; the arrays are
+ *     written only on success.
+ */
+HIFA4_API int hifa4_calibration_save(const char* path, int Hkv, int d, float alpha, const float* s, const float* sinv);
+HIFA4_API int hifa4_calibration_load(const char* path, int* Hkv, int* d, float* alpha, float* s, float* sinv,
+                                     size_t capacity);
 
 /*
  * Smooth-QK application + 4-bit quantisation of Q and K (one launch):
@@ -177,12 +197,11 @@ HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, co
  * holding a visible key when causal):
  *   S      = Q_hat K_hat_j^T                     (4-bit tensor-core MMA, fp32 accumulate)
  *   m_new  = max(m, fp16_RN(RN(rowmax(S) * c))), c = RN(log2(e) / sqrt(d))
- *   P      = E(RN(fma(S, c, -m_new)))            (E: the library's deterministic exp2)
- *   P_hat  = 4-bit blocks of 16 keys, each block's scale sigma from E(fma(blockmax S, c,
- *            -m_new)); a score's code is the E2M1 rounding of y = 2^floor(z) (1 + frac z),
- *            z = 128u - 125 - 73/1024 on a 2^-10 grid, u = sat(S c/128 + (RN(-log2 sigma)
- *            - m_new + 125)/128): P / sigma evaluated in the log domain with a linear
- *            mantissa (rounding boundaries within 1% of the exact exponential's)
+ *   P      = E(RN(fma(S, c, -m_new)))            (E: the library's deterministic exp2,
+ *            a cubic fit of 2^x with relative error below 9e-5)
+ *   P_hat  = the 4-bit block quantiser applied to P, 16 consecutive keys per block:
+ *            sigma = E4M3_RN(RN(amax * RN(1/6))) with amax the block's largest P, code =
+ *            E2M1_RN(RN(P * RN(1/sigma)))
  *   alpha  = E(m - m_new)  (0 on the first tile)
  *   O      = alpha * O + P_hat V_hat_j           (4-bit MMA)
  *   r      = P_hat * 1                           (4-bit MMA against ones: P-Reordering)
@@ -196,6 +215,21 @@ HIFA4_API int hifa4_quantize_qkv(const void* q, const void* k, const void* v, co
 HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt, int B,
                              int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o, void* m_out,
                              void* l_out, int* status, cudaStream_t stream);
+
+/*
+ * Fast form of hifa4_attn_fwd_quantized (same arguments, outputs and errors) with an
+ * approximate P_hat code rule: the code of a score is the E2M1 rounding of
+ * y = 2^floor(z) (1 + frac z), z = 128u - 125 - 73/1024 on a 2^-10 grid,
+ * u = sat(S c/128 + (RN(-log2 sigma) - m_new + 125)/128), i.e. P / sigma evaluated in the
+ * log domain with a linear mantissa, whose E2M1 rounding boundaries lie within 1% of the
+ * exact ones (the lowest, between codes 0 and 1, 5% above it).  m, sigma and alpha are
+ * those of hifa4_attn_fwd_quantized, so m is identical; a few percent of the P_hat codes
+ * differ by one step, which changes l and O slightly (the tests and the benchmark report
+ * the rates).  It exists to measure what the exact rounding costs.
+ */
+HIFA4_API int hifa4_attn_fwd_quantized_fast(const hifa4_qtensor* q, const hifa4_qtensor* k, const hifa4_qtensor* vt,
+                                            int B, int Hq, int Hkv, int N, int d, int causal, int kv_tile, void* o,
+                                            void* m_out, void* l_out, int* status, cudaStream_t stream);
 
 /*
  * Ablation form of hifa4_attn_fwd_quantized (same arguments, outputs and errors, plus
@@ -212,8 +246,7 @@ HIFA4_API int hifa4_attn_fwd_quantized(const hifa4_qtensor* q, const hifa4_qtens
  *   two_level 1: a second-level scale for P: per row and kv tile a power of two 2^k,
  *                k = max(floor(log2 p_t) - 10, -40) with p_t the tile's largest block amax
  *                of P; block scale E4M3_RN(RN(amax * RN(1/6)) * 2^-k), P_hat = code *
- *                scale * 2^k, and the code rule's L(sigma) taken for the effective scale
- *                scale * 2^k.  Equal to two_level 0 wherever every one-level block scale
+ *                scale * 2^k, code = E2M1_RN(RN(P * RN(1/(scale * 2^k)))).  Equal to two_level 0 wherever every one-level block scale
  *                is a normal E4M3 value; keeps the blocks one level flushes to zero
  *                (amax <= 6 * 2^-10).  l is the FP16 recursion on sum P_hat computed by the
  *                tensor core in fp32, which the wider scale range can round.
@@ -285,7 +318,8 @@ HIFA4_API int hifa4_attn_fwd(const hifa4_qtensor* q, const hifa4_qtensor* k, con
  * Allocates nothing.  The first call on a device looks up the scratch array's device
  * address (cudaGetSymbolAddress), so make that first call before any stream capture.
  * All calls on a device share the scratch: calls whose GPU work may overlap (e.g. on
- * unordered streams) race on it.
+ * unordered streams) race on it.  The scratch address is cached per device for the life
+ * of the process: after a cudaDeviceReset this entry point must not be called again.
  */
 HIFA4_API int hifa4_attn_fwd_noalloc(const hifa4_qtensor* q, const hifa4_qtensor* k, const void* v,
                                      const int64_t v_strides[3], int B, int Hq, int Hkv, int N, int d, int causal,
@@ -300,30 +334,6 @@ HIFA4_API int hifa4_read_status(int* status, int clear, cudaStream_t stream);
 
 /* Wall-clock limit of every wait inside the kernels, in nanoseconds (default 2 s). */
 HIFA4_API void hifa4_set_wait_limit_ns(unsigned long long ns);
-
-/*
- * Test hook: mode 1 makes the attention kernel's loader skip kv tile 1, so its
- * consumers' bounded waits run out and the call reports HIFA4_ERR_TIMEOUT through the
- * status word without hanging.  0 (default) disables it.
- */
-HIFA4_API void hifa4_debug_set_injection(int mode);
-
-/*
- * Single-tile probes of the tensor-core path (test and debug exports).
- *   hifa4_probe_qk_tile: S[128][kv_tile] fp32 = Q_hat K_hat^T for one 128-row Q tile
- *     (codes [128][d/2], scale atoms d/64 x 512 B) and one kv_tile-row K tile (codes
- *     [kv_tile][d/2], scale atoms d/64 x 512 B, keys in atom rows 0..kv_tile-1).
- *   hifa4_probe_pv_tile: O[128][d] fp32 = P_hat V_hat and R[128] fp32 = P_hat * 1 for one
- *     P_hat tile (codes [128][kv_tile/2], atoms kv_tile/64 x 512 B) and one V^T tile
- *     (codes [d][kv_tile/2], atoms (kv_tile/64) x ceil(d/128) x 512 B).
- *   hifa4_probe_codec: for each x[i]: E2M1 code of x, E4M3 code of |x| and the library's
- *     exp2 E(x), computed by the device conversions the kernels use.
- */
-HIFA4_API int hifa4_probe_qk_tile(const void* q_codes, const void* q_scales, const void* k_codes, const void* k_scales,
-                        int d, int kv_tile, float* S, int* status, cudaStream_t stream);
-HIFA4_API int hifa4_probe_pv_tile(const void* p_codes, const void* p_scales, const void* vt_codes, const void* vt_scales,
-                        int d, int kv_tile, float* O, float* R, int* status, cudaStream_t stream);
-HIFA4_API int hifa4_probe_codec(const float* x, int n, uint8_t* e2m1, uint8_t* e4m3, float* exp2_out, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -23,6 +23,22 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, n), n
 
 
+def test_test_hooks_only_in_the_test_library(L):
+    # the product library carries no probe and no fault injection; the test library holds
+    # the product ABI plus every function include/hifa4_test.h declares
+    from bit_flashattention_b200 import hifa4_testhooks as th
+    T = th.lib()
+    hooks = th.declared_functions()
+    assert set(hooks) >= {"hifa4_test_attn_fwd_inject", "hifa4_probe_codec", "hifa4_probe_qk_tile",
+                          "hifa4_probe_pv_tile"}
+    for n in hooks:
+        assert hasattr(T, n), n
+        assert not hasattr(L, n), n
+    for n in hifa4.declared_functions():
+        assert hasattr(T, n), n
+    assert not hasattr(L, "hifa4_debug_set_injection")
+
+
 def test_status_strings(L):
     for code in range(7):
         assert hifa4.status_string(code).startswith("HIFA4_")
@@ -119,6 +135,32 @@ def test_attn_fwd_checks_the_attention_before_quantising_v(L):
     # a workspace too small for V^T
     assert L.hifa4_attn_fwd(ctypes.byref(q), ctypes.byref(k), p, st, 1, 2, 2, 128, 128, 1, 0, p, ws - 16, p, None,
                             None, status, None) == hifa4.ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_a_workload_beyond_its_scratch_before_any_cuda_call(L):
+    # the allocation-free entry point checks the V^T size against its fixed 16 MiB scratch
+    # first: on a machine without a GPU it answers UNSUPPORTED_SHAPE (a CUDA call would
+    # have produced UNSUPPORTED_DEVICE), with host dummy pointers
+    fn = L.hifa4_attn_fwd_noalloc
+    P, i = ctypes.c_void_p, ctypes.c_int
+    QP = ctypes.POINTER(hifa4._QT)
+    fn.argtypes = [QP, QP, P, P, i, i, i, i, i, i, i, P, P, P, P, P]
+    fn.restype = i
+    buf = np.zeros(1 << 12, np.uint8)
+    p = ctypes.c_void_p(((buf.ctypes.data + 15) // 16) * 16)
+    B, Hq, Hkv, N, d = 4, 32, 8, 16384, 128                  # V^T ~37 MB
+    assert L.hifa4_attn_workspace_bytes(B, Hkv, N, d) > (16 << 20)
+    qt = hifa4._QT(p, p, B, Hq, N, d, 0)
+    kt = hifa4._QT(p, p, B, Hkv, N, d, 0)
+    st = (ctypes.c_int64 * 3)(0, 0, d)
+    assert fn(ctypes.byref(qt), ctypes.byref(kt), p, st, B, Hq, Hkv, N, d, 1, 0, p, None, None, p,
+              None) == hifa4.ERR_UNSUPPORTED_SHAPE
+    # a workload that fits goes on to the device check, which fails here without a GPU
+    B, Hq, Hkv, N = 1, 4, 2, 1024
+    qt = hifa4._QT(p, p, B, Hq, N, d, 0)
+    kt = hifa4._QT(p, p, B, Hkv, N, d, 0)
+    assert fn(ctypes.byref(qt), ctypes.byref(kt), p, st, B, Hq, Hkv, N, d, 1, 0, p, None, None, p,
+              None) == hifa4.ERR_UNSUPPORTED_DEVICE
 
 
 def test_layout_permutations_roundtrip():

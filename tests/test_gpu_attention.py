@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from bit_flashattention_b200 import configs, gen, hifa4
+from bit_flashattention_b200 import configs, gen, hifa4, hifa4_testhooks as th
 from tests import gpu_common as gc
 
 pytestmark = pytest.mark.gpu
@@ -107,14 +107,23 @@ def test_timeout_is_reported_and_context_survives():
     w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=512)
     q, k, v = gen.inputs(w)
     qq, kq, vq, vt = gc.gpu_quantize(w, q, k, v, None, None)
-    hifa4.hifa4_set_wait_limit_ns(200_000_000)
-    hifa4.hifa4_debug_set_injection(1)
+    # the injection is an argument of the test library's entry point, with that library's
+    # own (shortened) wait limit: the product library's calls are untouched
+    th.set_wait_limit_ns(200_000_000)
     try:
-        _, _, _, code = gc.gpu_attention(w, qq, kq, vt)
+        st = hifa4.new_status("cuda")
+        th.attn_fwd_inject(qq, kq, vq, causal=w.causal, kv_tile=w.bc, inject=1, status=st)
+        code = hifa4.hifa4_read_status(st)
     finally:
-        hifa4.hifa4_debug_set_injection(0)
-        hifa4.hifa4_set_wait_limit_ns(2_000_000_000)
+        th.set_wait_limit_ns(2_000_000_000)
     assert code == hifa4.ERR_TIMEOUT
+    # without the injection the same test entry point is the plain forward
+    st = hifa4.new_status("cuda")
+    o1, m1, l1 = th.attn_fwd_inject(qq, kq, vq, causal=w.causal, kv_tile=w.bc, inject=0, status=st)
+    assert hifa4.hifa4_read_status(st) == hifa4.OK
+    o2, m2, l2, code2 = gc.gpu_attention(w, qq, kq, vt)
+    assert code2 == hifa4.OK
+    assert torch.equal(o1, o2) and torch.equal(m1, m2) and torch.equal(l1, l2)
     # the context is still usable and the next call is correct
     gc.assert_parity(gc.run_parity(w))
 

@@ -4,9 +4,10 @@ probes of the block-scaled FP4 tensor-core MMAs (the S accumulation probe fixes 
 fp32 accumulation model the oracle mirrors)."""
 import numpy as np
 import pytest
+import torch
 
 import oracle
-from bit_flashattention_b200 import configs, gen, hifa4
+from bit_flashattention_b200 import configs, gen, hifa4, hifa4_testhooks as th
 from tests import _layout, gpu_common as gc
 from tests.test_oracle_formats import _boundary_values
 
@@ -20,7 +21,7 @@ def test_device_codec_and_exp2_match_oracle():
                          np.arange(0xBF800000, 0xC0000000, 37, dtype=np.uint32).view(np.float32),
                          np.array([-np.inf, -127.0, -126.0, 0.0, -0.0], np.float32)])
     allx = np.concatenate([x, ex]).astype(np.float32)
-    e2, e4, e = hifa4.hifa4_probe_codec(gc.to_dev(allx))
+    e2, e4, e = th.probe_codec(gc.to_dev(allx))
     e2, e4, e = e2.cpu().numpy(), e4.cpu().numpy(), e.cpu().numpy()
     n = len(x)
     assert np.array_equal(e2[:n], oracle.e2m1_encode(x))
@@ -28,6 +29,33 @@ def test_device_codec_and_exp2_match_oracle():
     fin = np.isfinite(ax)
     assert np.array_equal(e4[:n][fin], oracle.e4m3_encode(ax[fin]))
     assert np.array_equal(e[n:].view(np.uint32), oracle.exp2(ex).view(np.uint32))
+
+
+def test_device_codec_exhaustive_over_every_finite_fp32():
+    # every finite fp32 bit pattern (both signs) through the device E2M1 conversion, and every
+    # finite non-negative one through the E4M3 conversion of the block scales, against the
+    # oracle's codec, in chunks of 2^28 patterns.  NaN and infinity are left out: the
+    # quantisers flag non-finite inputs instead of converting them, and the softmax weights
+    # are finite by construction.
+    chunk = 1 << 28
+    e2 = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    e4 = torch.empty(chunk, dtype=torch.uint8, device="cuda")
+    checked = 0
+    for start in range(0, 1 << 32, chunk):
+        g2, g4 = th.probe_codec_range(start, chunk, e2, e4)
+        g2, g4 = g2.cpu().numpy(), g4.cpu().numpy()
+        bits = np.arange(start, start + chunk, dtype=np.uint32)
+        x = bits.view(np.float32)
+        fin = np.isfinite(x)
+        ref2 = oracle.e2m1_encode(x[fin])
+        bad = np.flatnonzero(g2[fin] != ref2)
+        assert bad.size == 0, ("e2m1", [hex(int(b)) for b in bits[fin][bad[:5]]])
+        if start < 0x80000000:                       # |x| of the negative half repeats these
+            ref4 = oracle.e4m3_encode(x[fin])
+            bad = np.flatnonzero(g4[fin] != ref4)
+            assert bad.size == 0, ("e4m3", [hex(int(b)) for b in bits[fin][bad[:5]]])
+        checked += int(fin.sum())
+    assert checked == (1 << 32) - 2 * ((1 << 23) * 1)      # all but the 2 * 2^23 NaN/inf patterns
 
 
 @pytest.mark.parametrize("name,kw", [
@@ -136,7 +164,7 @@ def test_qk_mma_probe_accumulation_model(d, bc):
     for narrow in (True, False):
         qc, qs = _rand_tile(rng, 128, d, narrow)
         kc, ks = _rand_tile(rng, bc, d, narrow)
-        S = hifa4.hifa4_probe_qk_tile(gc.to_dev(qc), gc.to_dev(_atoms_rows(qs, 128, d)), gc.to_dev(kc),
+        S = th.probe_qk_tile(gc.to_dev(qc), gc.to_dev(_atoms_rows(qs, 128, d)), gc.to_dev(kc),
                                       gc.to_dev(_atoms_rows(ks, bc, d)), d, bc).cpu().numpy()
         exact = oracle.qk_scores(qc, qs, kc, ks, 2).astype(np.float64)
         rel = np.max(np.abs(S - exact) / np.maximum(np.abs(exact), 1e-30))
@@ -159,7 +187,7 @@ def test_pv_mma_probe(d, bc):
     vs = rng.integers(0x28, 0x48, (d, bc // 16), dtype=np.uint8)
     p_atoms = _layout.rows_scales_from_plain(ps[None, None], 1, 1, 128, bc)
     v_atoms = _layout.vt_scales_from_plain(vs[None, None], 1, 1, bc, d)
-    O, R = hifa4.hifa4_probe_pv_tile(gc.to_dev(pc), gc.to_dev(p_atoms), gc.to_dev(vc), gc.to_dev(v_atoms), d, bc)
+    O, R = th.probe_pv_tile(gc.to_dev(pc), gc.to_dev(p_atoms), gc.to_dev(vc), gc.to_dev(v_atoms), d, bc)
     O, R = O.cpu().numpy().astype(np.float64), R.cpu().numpy().astype(np.float64)
 
     def deq(c, s):

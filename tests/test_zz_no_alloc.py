@@ -2,8 +2,9 @@
 device memory (their memory is all handed out up front, or they must not block on
 cudaMalloc).  It keeps the 4-bit V^T in a fixed 16 MiB array inside the library instead
 of a caller workspace.  Called through the C ABI, on two different inputs in a row, it
-must give what hifa4_attn_fwd gives on the same inputs, and it must reject a workload
-whose scratch would not fit.  Collected last so that a failure here cannot hide others."""
+must give bit for bit what hifa4_attn_fwd gives on the same inputs (the same kernels run
+on the same operands; only the V^T buffer differs), and it must reject a workload whose
+scratch would not fit.  Collected last so that a failure here cannot hide others."""
 import ctypes
 
 import pytest
@@ -51,10 +52,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         assert code == hifa4.OK
         o, m, l = _call_noalloc(w, qq, kq, vt)
         torch.cuda.synchronize()
-        assert torch.equal(m.float(), m_ref.float()) and torch.equal(l.float(), l_ref.float())
-        diff = (o.float() - o_ref.float()).abs()
-        assert diff.max().item() <= gc.O_MAX_ABS
-        assert diff.mean().item() / o_ref.float().abs().mean().item() <= gc.O_MEAN_REL
+        assert torch.equal(m, m_ref) and torch.equal(l, l_ref)
+        assert torch.equal(o, o_ref)
 
 
 def test_noalloc_rejects_workload_beyond_its_scratch():
