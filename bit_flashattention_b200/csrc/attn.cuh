@@ -85,7 +85,7 @@ struct AttnCfg {
   static constexpr int NSW0 = (BC < D ? BC : D) / 32;
   static constexpr int NSW = NSW0 < HIFA4_MAX_NSW ? NSW0 : HIFA4_MAX_NSW, CW = BC / NSW;
   static_assert(NSW == 2 || NSW == 4, "softmax warpgroups");
-  static_assert(CW == 32 || CW == 64, "column split");
+  static_assert(CW == 32 || CW == 64 || CW == 128, "column split");
   static constexpr int NTHREADS = 96 + 128 * NSW;   // producer, QK^T issuer, PV issuer, softmax
 };
 
@@ -456,6 +456,13 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
     const int col0 = wg * CW;
     const float c = p.c;
     const float c7 = c * 0.0078125f;
+    // this thread's byte offsets in a P_hat buffer (swizzled K-major rows) and in its scale atoms
+    uint32_t p_off[CW / 32];
+#pragma unroll
+    for (int q = 0; q < CW / 32; ++q) p_off[q] = swz_offset(row, col0 / 32 + q, C::PROW);
+    // one scale atom per 64 columns: CW / 64 atoms (CW = 128), or a part of one
+    constexpr int NATOM = CW >= 64 ? CW / 64 : 1;
+    const uint32_t psf_off = 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
     // Epilogue of a unit whose last tile is gl: read R and O of that tile's PV, release
     // them (o_free), then O / l -> bf16 (decode: the unnormalised fp32 O and l of the
     // split's partial).  It runs after the next unit's first tile, which touches neither O
@@ -624,44 +631,48 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           pmax[bl + 1] = e2.y;
         }
         uint32_t words[CW / 8];
-        uint32_t sfw = 0;
+        uint64_t sfw = 0;                    // the NB scale bytes, block bl in byte bl
         float part = 0.0f;                   // ablation kernels: this warpgroup's sum of P
+        // the blocks' scales and codes
+        {
 #pragma unroll
-        for (int bl = 0; bl < NB; ++bl) {
-          float sarg = __fmul_rn(pmax[bl], kSixth);
-          if constexpr (SUMP) sarg = __fmul_rn(sarg, kinv);
-          const uint32_t sc = cvt_e4m3(sarg);
-          sfw |= sc << (8 * bl);
-          if constexpr (FAST) {
-            // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
-            const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
+          for (int bl = 0; bl < NB; ++bl) {
+            float sarg = __fmul_rn(pmax[bl], kSixth);
+            if constexpr (SUMP) sarg = __fmul_rn(sarg, kinv);
+            const uint32_t sc = cvt_e4m3(sarg);
+            sfw |= (uint64_t)sc << (8 * bl);
+            if constexpr (FAST) {
+              // B = (L(sigma) - m + 125) / 128; L(0) = -inf makes every code of the block 0
+              const float B = __fmul_rn(__fadd_rn(__fsub_rn(rtab[sc], mnew), 125.0f), 0.0078125f);
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-              float2 y[4];
+              for (int h8 = 0; h8 < 2; ++h8) {
+                float2 y[4];
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int e = bl * 16 + h8 * 8 + 2 * k;
-                y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
+                for (int k = 0; k < 4; ++k) {
+                  const int e = bl * 16 + h8 * 8 + 2 * k;
+                  y[k] = phat_pair(make_float2(fma_sat(s[e], c7, B), fma_sat(s[e + 1], c7, B)));
+                }
+                words[2 * bl + h8] = encode8_pairs(y);
               }
-              words[2 * bl + h8] = encode8_pairs(y);
-            }
-          } else {
-            // code = E2M1_RN(RN(P * R)), R = RN(1/sigma) (0 for sigma = 0); with the
-            // two-level scale R = RN(1/(sigma 2^k)) = RN(1/sigma) 2^-k, exact
-            float R = rtab[sc];
-            if constexpr (SUMP) R = __fmul_rn(R, kinv);
-            const float2 R2 = make_float2(R, R);
+            } else {
+              // code = E2M1_RN(RN(P * R)), R = RN(1/sigma) (0 for sigma = 0); with the
+              // two-level scale R = RN(1/(sigma 2^k)) = RN(1/sigma) 2^-k, exact
+              float R = rtab[sc];
+              if constexpr (SUMP) R = __fmul_rn(R, kinv);
+              const float2 R2 = make_float2(R, R);
 #pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-              float2 y[4];
+              for (int h8 = 0; h8 < 2; ++h8) {
+                float2 y[4];
 #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int e = bl * 16 + h8 * 8 + 2 * k;
-                const float2 e2 = exp2_own2(__ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2));
-                if constexpr (SUMP) part = __fadd_rn(__fadd_rn(part, e2.x), e2.y);
-                y[k] = __fmul2_rn(e2, R2);
+                for (int k = 0; k < 4; ++k) {
+                  const int e = bl * 16 + h8 * 8 + 2 * k;
+                  const float2 x2 = __ffma2_rn(make_float2(s[e], s[e + 1]), c2, negm2);
+                  const float2 e2 = exp2_own2(x2);
+                  if constexpr (SUMP) part = __fadd_rn(__fadd_rn(part, e2.x), e2.y);
+                  y[k] = __fmul2_rn(e2, R2);
+                }
+                words[2 * bl + h8] = encode8_pairs(y);
               }
-              words[2 * bl + h8] = encode8_pairs(y);
             }
           }
         }
@@ -677,11 +688,12 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         uint8_t* pbuf = sP(pb);
 #pragma unroll
         for (int q = 0; q < CW / 32; ++q)
-          *reinterpret_cast<uint4*>(pbuf + swz_offset(row, col0 / 32 + q, C::PROW)) =
+          *reinterpret_cast<uint4*>(pbuf + p_off[q]) =
               make_uint4(words[4 * q], words[4 * q + 1], words[4 * q + 2], words[4 * q + 3]);
-        {
-          uint8_t* atom = sPsf(pb) + 512 * (col0 / 64) + sf_atom_offset(row, (col0 % 64) / 16);
-          if (NB == 4) *reinterpret_cast<uint32_t*>(atom) = sfw;
+#pragma unroll
+        for (int a = 0; a < NATOM; ++a) {
+          uint8_t* atom = sPsf(pb) + psf_off + 512 * a;
+          if (NB >= 4) *reinterpret_cast<uint32_t*>(atom) = (uint32_t)(sfw >> (32 * a));
           else *reinterpret_cast<uint16_t*>(atom) = (uint16_t)sfw;
         }
         fence_proxy_async_smem();

@@ -180,18 +180,58 @@ void fill_neg_log2_scales(float* t) {
 // The streaming quantiser (k_quant_stream) over Q and K row chunks (4096 / d rows each)
 // and V chunks (32 tokens each); the callers set each struct's `units` in those chunks,
 // 0 for a tensor that is not quantised.
-int launch_quant_stream(const QuantRowsArgs& qa, const QuantRowsArgs& ka, const QuantVtArgs& va, int d, int* status,
-                        cudaStream_t stream) {
-  const int units = qa.units + ka.units + va.units;
-  switch (d) {
-    case 64: k_quant_stream<64><<<resident_grid(k_quant_stream<64>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-    case 128: k_quant_stream<128><<<resident_grid(k_quant_stream<128>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-    default: k_quant_stream<256><<<resident_grid(k_quant_stream<256>, 256, units), 256, 0, stream>>>(qa, ka, va, status); break;
-  }
+template <int D, bool ROPE>
+int launch_quant_stream_d(const QuantRowsArgs& qa, const QuantRowsArgs& ka, const QuantVtArgs& va, int* status,
+                          cudaStream_t stream) {
+  // multiply-shift constants of the chunk index splits (chunks per head, heads, group size)
+  auto fd = [](int v) { return make_fastdiv((uint32_t)(v > 0 ? v : 1)); };
+  StreamDivs dv;
+  dv.q_chunks = fd(qa.N / StreamCfg<D>::RC);
+  dv.q_heads = fd(qa.H);
+  dv.q_group = fd(qa.Hkv > 0 ? qa.H / qa.Hkv : 1);
+  dv.k_chunks = fd(ka.N / StreamCfg<D>::RC);
+  dv.k_heads = fd(ka.H);
+  dv.k_group = fd(ka.Hkv > 0 ? ka.H / ka.Hkv : 1);
+  dv.v_chunks = fd(va.N / StreamCfg<D>::TV);
+  dv.v_heads = fd(va.H);
+  constexpr uint32_t smem = StreamCfg<D>::SMEM;
+  // shared-memory attribute and resident CTAs (at most 3, with RoPE 2: the kernel's register bound),
+  // set up once per instance (thread-safe static initialisation)
+  static const int per_sm = [] {
+    if (!set_smem(k_quant_stream<D, ROPE>, smem)) return 0;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_quant_stream<D, ROPE>, 256, smem) != cudaSuccess || n <= 0)
+      n = 1;
+    const int cap_regs = ROPE ? 2 : 3;
+    return n < cap_regs ? n : cap_regs;
+  }();
+  if (per_sm == 0) return HIFA4_ERR_CUDA;
+  const long long units = (long long)qa.units + ka.units + va.units;
+  const long long cap = (long long)per_sm * num_sms();
+  k_quant_stream<D, ROPE><<<(unsigned)(units < cap ? units : cap), 256, smem, stream>>>(qa, ka, va, dv, status,
+                                                                                        g_wait_ns);
   return cuda_status(cudaGetLastError());
 }
 
-int stream_row_chunks(int B, int H, int N, int d) { return B * H * (N / (4096 / d)); }
+int launch_quant_stream(const QuantRowsArgs& qa, const QuantRowsArgs& ka, const QuantVtArgs& va, int d, int* status,
+                        cudaStream_t stream, bool rope = false) {
+  if ((long long)qa.units + ka.units + va.units == 0) return HIFA4_OK;
+  if (rope) {
+    switch (d) {
+      case 64: return launch_quant_stream_d<64, true>(qa, ka, va, status, stream);
+      case 128: return launch_quant_stream_d<128, true>(qa, ka, va, status, stream);
+      default: return launch_quant_stream_d<256, true>(qa, ka, va, status, stream);
+    }
+  }
+  switch (d) {
+    case 64: return launch_quant_stream_d<64, false>(qa, ka, va, status, stream);
+    case 128: return launch_quant_stream_d<128, false>(qa, ka, va, status, stream);
+    default: return launch_quant_stream_d<256, false>(qa, ka, va, status, stream);
+  }
+}
+
+// chunks of the streaming quantiser: 16 KB of bf16 input each (8192 / d rows or tokens)
+int stream_row_chunks(int B, int H, int N, int d) { return B * H * (N / (8192 / d)); }
 
 // Decode / split-KV launch parameters (see AttnParams).
 struct DecodeSpec {
@@ -488,20 +528,14 @@ int hifa4_quantize_qk_rope(const void* q, const void* k, const int64_t q_strides
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || N <= 0 || N % 128 || !d_ok(d)) return HIFA4_ERR_UNSUPPORTED_SHAPE;
   if (!qt_ok(q_out, B, Hq, N, d, 0) || !qt_ok(k_out, B, Hkv, N, d, 0)) return HIFA4_ERR_INVALID_ARG;
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
-  const int rows = d == 256 ? 64 : 128;
   QuantRowsArgs qa{static_cast<const __nv_bfloat16*>(q), q_strides[0], q_strides[1], q_strides[2], Hq, Hkv, N, s,
                    rope_cos, rope_sin, 0, 0, static_cast<uint8_t*>(q_out->codes), static_cast<uint8_t*>(q_out->scales),
-                   B * Hq * (N / rows)};
+                   stream_row_chunks(B, Hq, N, d)};
   QuantRowsArgs ka{static_cast<const __nv_bfloat16*>(k), k_strides[0], k_strides[1], k_strides[2], Hkv, Hkv, N, sinv,
                    rope_cos, rope_sin, 0, 0, static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales),
-                   B * Hkv * (N / rows)};
-  const int units = qa.units + ka.units;
-  switch (d) {
-    case 64: k_quant_rows_rope<64><<<resident_grid(k_quant_rows_rope<64>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-    case 128: k_quant_rows_rope<128><<<resident_grid(k_quant_rows_rope<128>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-    default: k_quant_rows_rope<256><<<resident_grid(k_quant_rows_rope<256>, 256, units), 256, 0, stream>>>(qa, ka, status); break;
-  }
-  return cuda_status(cudaGetLastError());
+                   stream_row_chunks(B, Hkv, N, d)};
+  QuantVtArgs va{};
+  return launch_quant_stream(qa, ka, va, d, status, stream, true);
 }
 
 int hifa4_rope_table(double theta, int pos0, int N, int d, float* cos_out, float* sin_out) {
@@ -526,7 +560,7 @@ int hifa4_quantize_v(const void* v, const int64_t v_strides[3], int B, int Hkv, 
   if (!device_ok()) return HIFA4_ERR_UNSUPPORTED_DEVICE;
   QuantRowsArgs none{};
   QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
-                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
+                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), stream_row_chunks(B, Hkv, N, d)};
   return launch_quant_stream(none, none, va, d, status, stream);
 }
 
@@ -548,7 +582,7 @@ int hifa4_quantize_qkv(const void* q, const void* k, const void* v, const int64_
                    nullptr, nullptr, 0, 0,
                    static_cast<uint8_t*>(k_out->codes), static_cast<uint8_t*>(k_out->scales), stream_row_chunks(B, Hkv, N, d)};
   QuantVtArgs va{static_cast<const __nv_bfloat16*>(v), v_strides[0], v_strides[1], v_strides[2], Hkv, N,
-                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), B * Hkv * (N / 32)};
+                 static_cast<uint8_t*>(vt_out->codes), static_cast<uint8_t*>(vt_out->scales), stream_row_chunks(B, Hkv, N, d)};
   return launch_quant_stream(qa, ka, va, d, status, stream);
 }
 

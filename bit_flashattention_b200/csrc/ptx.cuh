@@ -55,7 +55,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete.  Gives up after `limit_ns` of
 // wall time (checked every 256 polls) or as soon as another role raised `*abort`; on
-// giving up it ORs ST_TIMEOUT into the status word and returns false.
+// giving up it ORs ST_TIMEOUT into the status word and returns false.  (A suspend-time
+// hint on the poll was measured slower for the attention kernel.)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;

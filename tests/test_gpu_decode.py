@@ -68,10 +68,13 @@ def test_decode_matches_oracle(case):
     qc, qs = oracle.quantize_rows(oracle.pack_decode_q(q, Hkv), Hkv, s)
     kc, ks = oracle.quantize_rows(k, Hkv, sinv)
     vc, vs = oracle.quantize_vt(v)
-    # the packed query and the K cache are bit-exact
+    # the packed query and the 4-bit K and V^T cache are bit-exact, codes and scales
     assert np.array_equal(qp.codes.cpu().numpy().reshape(qc.shape), qc)
     assert np.array_equal(_layout.rows_scales_to_plain(qp.scales.cpu().numpy(), B, Hkv, 128, d), qs)
     assert np.array_equal(kq.codes.cpu().numpy().reshape(kc.shape), kc)
+    assert np.array_equal(_layout.rows_scales_to_plain(kq.scales.cpu().numpy(), B, Hkv, Nk, d), ks)
+    assert np.array_equal(vq.codes.cpu().numpy().reshape(vc.shape), vc)
+    assert np.array_equal(_layout.vt_scales_to_plain(vq.scales.cpu().numpy(), B, Hkv, Nk, d), vs)
 
     bc = kv_tile if kv_tile else 128
     ref = oracle.attn_decode(qc, qs, kc, ks, vc, vs, G=G, nq=nq, bc=bc, nsplit=nsplit)

@@ -23,8 +23,12 @@ def _pre_rope(rng, B, H, N, d, outliers=0):
 
 
 def _check_rows(qt, codes, scales, B, H, N, d):
-    assert np.array_equal(qt.codes.cpu().numpy().reshape(codes.shape), codes)
-    assert np.array_equal(_layout.rows_scales_to_plain(qt.scales.cpu().numpy(), B, H, N, d), scales)
+    got = qt.codes.cpu().numpy().reshape(codes.shape)
+    bad = np.argwhere(got != codes)
+    assert bad.size == 0, (len(bad), bad[:8].tolist(), got[tuple(bad[:4].T)].tolist(), codes[tuple(bad[:4].T)].tolist())
+    gs = _layout.rows_scales_to_plain(qt.scales.cpu().numpy(), B, H, N, d)
+    bad = np.argwhere(gs != scales)
+    assert bad.size == 0, (len(bad), bad[:8].tolist())
 
 
 @pytest.mark.parametrize("d,smooth", [(64, False), (128, True), (128, False), (256, True)])
