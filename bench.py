@@ -407,6 +407,27 @@ def run_gpu(args):
     # the secondary measurements below run on the rank's first block of heads
     c0 = blk[0]
 
+    # the quantiser alone (back to back over the rotated inputs): inside the step it also
+    # absorbs the DRAM write-back of the previous attention's O, m, l (34 MB at Qwen 4k),
+    # which the attention leaves in L2
+    n_q = max(20, min(args.steps, 400))
+    q0 = torch.cuda.Event(enable_timing=True)
+    q1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    q0.record(stream)
+    for i in range(n_q):
+        qt, kt, vt = sets[i % N_SETS]
+        for c in blk:
+            hifa4.hifa4_quantize_qkv(views(qt, c["b0"], c["b1"], c["g0"] * G, c["g1"] * G),
+                                     views(kt, c["b0"], c["b1"], c["g0"], c["g1"]),
+                                     views(vt, c["b0"], c["b1"], c["g0"], c["g1"]), c["s"], c["sinv"], status=st,
+                                     out=(c["q"][0], c["k"][0], c["v"][0]))
+    q1.record(stream)
+    torch.cuda.synchronize()
+    k_quant_alone = q0.elapsed_time(q1) / n_q
+    if hifa4.hifa4_read_status(st) != hifa4.OK:
+        raise RuntimeError("quantiser-alone loop reported an error")
+
     def in0(i):
         qt, kt, vt = sets[i % N_SETS]
         return (views(qt, c0["b0"], c0["b1"], c0["g0"] * G, c0["g1"] * G), views(kt, c0["b0"], c0["b1"], c0["g0"], c0["g1"]),
@@ -503,6 +524,7 @@ def run_gpu(args):
     k_attn = reduce_max(k_attn, dist, device)
     k_quant = reduce_max(k_quant, dist, device)
     k_rope = reduce_max(k_rope, dist, device)
+    k_quant_alone = reduce_max(k_quant_alone, dist, device)
     decode = measure_decode(hifa4, torch, device, max(20, min(args.steps, 200)), dist)
     fp4 = measure_fp4_peak(torch, device, local, dist)
     flops_all = reduce_sum(flops, dist, device)
@@ -547,6 +569,11 @@ def run_gpu(args):
         "attn_kernel_tflops": round(achieved, 2),
         "quantize_qkv_gbs": round(quant_bytes / (k_quant * 1e-3) / 1e9, 1),
         "quantize_qkv_frac_hbm": round(quant_bytes / (k_quant * 1e-3) / 1e9 / hbm, 3),
+        "quantize_qkv_alone": {"us": round(k_quant_alone * 1e3, 2),
+                               "gbs": round(quant_bytes / (k_quant_alone * 1e-3) / 1e9, 1),
+                               "frac_hbm": round(quant_bytes / (k_quant_alone * 1e-3) / 1e9 / hbm, 3),
+                               "note": "quantiser launches back to back over the rotated inputs; inside the step "
+                                       "(kernels_us) it also absorbs the previous attention's O write-back"},
         "decode": decode,
         "fast_phat": fast,
         "quantize_qk_rope": {"us": round(k_rope * 1e3, 2), "launches": n_rope,
