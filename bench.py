@@ -29,9 +29,11 @@ WORKLOAD = "qwen3-8b-4k"
 N_SETS = 6                      # rotated input sets: 6 x ~50 MB of bf16 inputs > 126 MB L2
 FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of one attention launch on qwen3-8b-4k from an ncu capture of
-# the current kernel (dram__bytes_read.sum + dram__bytes_write.sum), or None when the
-# kernel has changed since the counters were taken.
-ATTN_TRAFFIC_BYTES = None
+# the current kernel (dram__bytes_read.sum + dram__bytes_write.sum = 14,224,640 + 42,496,
+# profiles/attn_fwd_qwen3-8b-4k.md), or None when the kernel has changed since the
+# counters were taken.  O, m and l (34.1 MB) are still in L2 when the launch ends, so they
+# are written back to DRAM during the next kernel and do not appear in this figure.
+ATTN_TRAFFIC_BYTES = 14267136
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 
@@ -540,6 +542,9 @@ def run_gpu(args):
     # algorithmic HBM bytes of one attention launch: 4-bit Q, K, V^T (codes + scales) read,
     # bf16 O and fp16 m, l written
     # (summed over the rank's blocks of heads)
+    # the captured traffic is that of one launch over the whole qwen3-8b-4k call
+    whole_call = WORKLOAD == "qwen3-8b-4k" and len(blocks) == 1 and blocks[0][1] - blocks[0][0] == w.B \
+        and blocks[0][2] == 0 and blocks[0][3] == w.Hkv
     attn_bytes = sum((b1 - b0) * ((g1 - g0) * (G + 2) * N * d * (0.5 + 1 / 16) + (g1 - g0) * G * N * (2 * d + 4))
                      for b0, b1, g0, g1 in blocks)
     quant_bytes = sum((b1 - b0) * (g1 - g0) * (G + 2) * N * d * (2 + 0.5 + 1 / 16) for b0, b1, g0, g1 in blocks)
@@ -584,7 +589,7 @@ def run_gpu(args):
                                      "the fp32 angle tables stay in L2"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
-                     "traffic": ATTN_TRAFFIC_BYTES if WORKLOAD == "qwen3-8b-4k" else None,
+                     "traffic": ATTN_TRAFFIC_BYTES if whole_call else None,
                      "algorithmic_bytes": attn_bytes,
                      "frac_of_bf16x4": round(achieved / fp4_nominal, 4),
                      "peak_source": f"measured: own FP4 MMA loop, burst (fp4_peak_measured); {src} bf16 burst x "
