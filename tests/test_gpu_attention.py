@@ -42,6 +42,12 @@ def test_parity_full_size_sampled_rows(name):
     gc.assert_parity(gc.run_parity(w, rows, check_quant=False))
 
 
+def test_parity_full_size_128_key_tiles_sampled_rows():
+    # the full Qwen3-8B-shaped 4k call at 128-key tiles (32 score columns per softmax warp)
+    w = configs.scaled(configs.get("qwen3-8b-4k"), bc=128)
+    gc.assert_parity(gc.run_parity(w, gen.sample_rows(w, per_head=4), check_quant=False))
+
+
 EDGE = [
     ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=128, bc=128)),                 # one query tile, one kv tile
     ("qwen3-8b-4k", dict(Hq=2, Hkv=1, N=128, bc=128, causal=False)),
@@ -103,8 +109,9 @@ def test_strided_value_input():
     gc.assert_parity(stats)
 
 
-def test_timeout_is_reported_and_context_survives():
-    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=512)
+@pytest.mark.parametrize("bc", [256, 128])
+def test_timeout_is_reported_and_context_survives(bc):
+    w = configs.scaled(configs.get("qwen3-8b-4k"), Hq=2, Hkv=1, N=512, bc=bc)
     q, k, v = gen.inputs(w)
     qq, kq, vq, vt = gc.gpu_quantize(w, q, k, v, None, None)
     # the injection is an argument of the test library's entry point, with that library's
