@@ -29,10 +29,11 @@ WORKLOAD = "qwen3-8b-4k"
 N_SETS = 6                      # rotated input sets: 6 x ~50 MB of bf16 inputs > 126 MB L2
 FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of one attention launch on qwen3-8b-4k from an ncu capture of
-# the current kernel (dram__bytes_read.sum + dram__bytes_write.sum = 14,224,640 + 42,496,
-# profiles/attn_fwd_qwen3-8b-4k.md), or None when the kernel has changed since the
-# counters were taken.  O, m and l (34.1 MB) are still in L2 when the launch ends, so they
-# are written back to DRAM during the next kernel and do not appear in this figure.
+# the current kernel (`--set full`, the first timed launch of this script's default run:
+# dram__bytes_read.sum 14,224,640 + dram__bytes_write.sum 42,496), or None when the kernel
+# has changed since the counters were taken.  O, m and l (34.1 MB) are still in L2 when the
+# launch ends, so they are written back to DRAM during the next kernel and do not appear
+# in this figure.
 ATTN_TRAFFIC_BYTES = 14267136
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
@@ -409,24 +410,48 @@ def run_gpu(args):
     # the secondary measurements below run on the rank's first block of heads
     c0 = blk[0]
 
-    # the quantiser alone (back to back over the rotated inputs): inside the step it also
-    # absorbs the DRAM write-back of the previous attention's O, m, l (34 MB at Qwen 4k),
-    # which the attention leaves in L2
-    n_q = max(20, min(args.steps, 400))
-    q0 = torch.cuda.Event(enable_timing=True)
-    q1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    q0.record(stream)
-    for i in range(n_q):
+    def graph_time(launch, n, reps):
+        """Average device time (ms) of launch(i) for i = 0..n-1, captured once in a CUDA graph
+        and replayed `reps` times, so the launch rate of the Python binding does not set the
+        time; a plain launch loop when the capture fails.  Returns (ms, description)."""
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for i in range(n):
+                    launch(i)
+            graph.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            del graph
+            how = f"one CUDA graph of {n} launches, replayed {reps} times"
+        except RuntimeError as e:
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(n * reps):
+                launch(i)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            how = f"Python launch loop (graph capture failed: {str(e)[:80]})"
+        return e0.elapsed_time(e1) / (n * reps), how
+
+    # the quantiser alone, back to back over the rotated inputs.  Inside the step the kernel
+    # also absorbs the DRAM write-back of the previous attention's O, m, l (34 MB at Qwen
+    # 4k), which the attention leaves in L2.
+    def quant_set(i):
         qt, kt, vt = sets[i % N_SETS]
         for c in blk:
             hifa4.hifa4_quantize_qkv(views(qt, c["b0"], c["b1"], c["g0"] * G, c["g1"] * G),
                                      views(kt, c["b0"], c["b1"], c["g0"], c["g1"]),
                                      views(vt, c["b0"], c["b1"], c["g0"], c["g1"]), c["s"], c["sinv"], status=st,
                                      out=(c["q"][0], c["k"][0], c["v"][0]))
-    q1.record(stream)
-    torch.cuda.synchronize()
-    k_quant_alone = q0.elapsed_time(q1) / n_q
+    reps = max(4, min(args.steps, 400) // N_SETS)
+    k_quant_alone, quant_alone_how = graph_time(quant_set, N_SETS, reps)
     if hifa4.hifa4_read_status(st) != hifa4.OK:
         raise RuntimeError("quantiser-alone loop reported an error")
 
@@ -441,18 +466,12 @@ def run_gpu(args):
     rc, rs = hifa4.hifa4_rope_table(w.rope_theta or 1e4, N, d)
     rc = torch.from_numpy(rc).to(device)
     rs = torch.from_numpy(rs).to(device)
-    n_rope = max(20, min(args.steps, 400))
+    def rope_set(i):
+        hifa4.hifa4_quantize_qk_rope(in0(i)[0], in0(i)[1], rc, rs, s0, sinv0, status=st, out=(qq[0], kq[0]))
     for i in range(3):
-        hifa4.hifa4_quantize_qk_rope(in0(i)[0], in0(i)[1], rc, rs, s0, sinv0, status=st, out=(qq[0], kq[0]))
-    r0 = torch.cuda.Event(enable_timing=True)
-    r1 = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    r0.record(stream)
-    for i in range(n_rope):
-        hifa4.hifa4_quantize_qk_rope(in0(i)[0], in0(i)[1], rc, rs, s0, sinv0, status=st, out=(qq[0], kq[0]))
-    r1.record(stream)
-    torch.cuda.synchronize()
-    k_rope = r0.elapsed_time(r1) / n_rope
+        rope_set(i)
+    k_rope, rope_how = graph_time(rope_set, N_SETS, reps)
+    n_rope = N_SETS * reps
     if hifa4.hifa4_read_status(st) != hifa4.OK:
         raise RuntimeError("fused RoPE quantiser reported an error")
 
@@ -577,11 +596,12 @@ def run_gpu(args):
         "quantize_qkv_alone": {"us": round(k_quant_alone * 1e3, 2),
                                "gbs": round(quant_bytes / (k_quant_alone * 1e-3) / 1e9, 1),
                                "frac_hbm": round(quant_bytes / (k_quant_alone * 1e-3) / 1e9 / hbm, 3),
+                               "launched_as": quant_alone_how,
                                "note": "quantiser launches back to back over the rotated inputs; inside the step "
                                        "(kernels_us) it also absorbs the previous attention's O write-back"},
         "decode": decode,
         "fast_phat": fast,
-        "quantize_qk_rope": {"us": round(k_rope * 1e3, 2), "launches": n_rope,
+        "quantize_qk_rope": {"us": round(k_rope * 1e3, 2), "launches": n_rope, "launched_as": rope_how,
                              "gbs": round(rope_bytes / (k_rope * 1e-3) / 1e9, 1),
                              "frac_hbm": round(rope_bytes / (k_rope * 1e-3) / 1e9 / hbm, 3),
                              "algorithmic_bytes": rope_bytes,

@@ -583,17 +583,22 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
           for (int q = 0; q < CW; ++q)
             if (j * BC + col0 + q > pos) s[q] = -INFINITY;
         }
+        // block maxima as a 3-input-max tree (depth 3), then the row part over the blocks
         float bmax[NB];
 #pragma unroll
         for (int bl = 0; bl < NB; ++bl) {
-          float m = s[bl * 16];
-#pragma unroll
-          for (int e = 1; e < 15; e += 2) m = fmax3(m, s[bl * 16 + e], s[bl * 16 + e + 1]);
-          bmax[bl] = fmaxf(m, s[bl * 16 + 15]);
+          const float* x = s + bl * 16;
+          const float u0 = fmax3(fmax3(x[0], x[1], x[2]), fmax3(x[3], x[4], x[5]), fmax3(x[6], x[7], x[8]));
+          const float u1 = fmax3(fmax3(x[9], x[10], x[11]), fmax3(x[12], x[13], x[14]), x[15]);
+          bmax[bl] = fmaxf(u0, u1);
         }
         float lmax = bmax[0];
+        if constexpr (NB == 4) {
+          lmax = fmaxf(fmax3(bmax[0], bmax[1], bmax[2]), bmax[3]);
+        } else {
 #pragma unroll
-        for (int bl = 1; bl < NB; ++bl) lmax = fmaxf(lmax, bmax[bl]);
+          for (int bl = 1; bl < NB; ++bl) lmax = fmaxf(lmax, bmax[bl]);
+        }
         // combine the partial row maxima of the NSW warpgroups (double-buffered by parity)
         float* xm = xmax + (g & 1) * (C::NSW * 128);
         xm[wg * 128 + row] = lmax;
@@ -603,9 +608,10 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
         float mnew = m_run;
         if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
-        // alpha = E(m - m_new): 0 on the first tile, exactly E(0) = 1 when the max is unchanged
-        const float alpha =
-            (m_run == -INFINITY) ? 0.0f : (mnew == m_run ? 1.0f : exp2_own(__fsub_rn(m_run, mnew)));
+        // alpha = E(m - m_new), without branches: on the first tile m = -inf and the argument
+        // is -inf (or NaN when m_new is -inf too), which E clamps to -127, so alpha = E(-127) = 0;
+        // when the max is unchanged the argument is 0 and alpha = E(0) = 1 exactly
+        const float alpha = exp2_own(__fsub_rn(m_run, mnew));
         const float negm = -mnew;
         const float2 c2 = make_float2(c, c), negm2 = make_float2(negm, negm);
         // O is rescaled by alpha_o: alpha, times 2^(k_prev - k) with the two-level scale
