@@ -603,11 +603,15 @@ __global__ void __launch_bounds__(AttnCfg<D, BC>::NTHREADS, 1)
         float* xm = xmax + (g & 1) * (C::NSW * 128);
         xm[wg * 128 + row] = lmax;
         named_bar(1 + q4, 32 * C::NSW);
-        float rmax = xm[row];
-#pragma unroll
-        for (int w2 = 1; w2 < C::NSW; ++w2) rmax = fmaxf(rmax, xm[w2 * 128 + row]);
-        float mnew = m_run;
-        if (rmax != -INFINITY) mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
+        float rmax;
+        if constexpr (C::NSW == 4) {
+          rmax = fmaxf(fmax3(xm[row], xm[128 + row], xm[256 + row]), xm[384 + row]);
+        } else {
+          rmax = fmaxf(xm[row], xm[128 + row]);
+        }
+        // m_new = max(m, fp16(RN(rowmax * c))); a row with no visible key keeps m (-inf * c
+        // rounds to -inf)
+        const float mnew = fmaxf(m_run, f16_round(__fmul_rn(rmax, c)));
         // alpha = E(m - m_new), without branches: on the first tile m = -inf and the argument
         // is -inf (or NaN when m_new is -inf too), which E clamps to -127, so alpha = E(-127) = 0;
         // when the max is unchanged the argument is 0 and alpha = E(0) = 1 exactly
