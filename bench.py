@@ -30,11 +30,11 @@ N_SETS = 6                      # rotated input sets: 6 x ~50 MB of bf16 inputs 
 FP4_OVER_BF16 = 4.0             # nominal dense FP4 / BF16 tensor throughput ratio (9 / 2.25 PFLOP/s)
 # DRAM bytes (read + write) of one attention launch on qwen3-8b-4k from an ncu capture of
 # the current kernel (`--set full`, the first timed launch of this script's default run:
-# dram__bytes_read.sum 14,224,640 + dram__bytes_write.sum 42,496), or None when the kernel
+# dram__bytes_read.sum 14,218,240 + dram__bytes_write.sum 42,240), or None when the kernel
 # has changed since the counters were taken.  O, m and l (34.1 MB) are still in L2 when the
 # launch ends, so they are written back to DRAM during the next kernel and do not appear
 # in this figure.
-ATTN_TRAFFIC_BYTES = 14267136
+ATTN_TRAFFIC_BYTES = 14260480
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 

@@ -419,10 +419,12 @@ __global__ void __launch_bounds__(DecTCfg::NTHREADS, NQ == 16 ? 2 : 3)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int qq = q + e;
-            float mn = m_run[qq];
-            if (rm[e] != -INFINITY) mn = fmaxf(m_run[qq], f16_round(__fmul_rn(rm[e], c)));
+            // branch-free: a row with no visible key keeps m (-inf * c rounds to -inf); E clamps
+            // the first tile's argument (-inf, or NaN when m_new is -inf too) to -127, so
+            // alpha = 0 there, and alpha = E(0) = 1 exactly when the max is unchanged
+            const float mn = fmaxf(m_run[qq], f16_round(__fmul_rn(rm[e], c)));
             mnew[qq] = mn;
-            alpha[qq] = (m_run[qq] == -INFINITY) ? 0.0f : (mn == m_run[qq] ? 1.0f : exp2_own(__fsub_rn(m_run[qq], mn)));
+            alpha[qq] = exp2_own(__fsub_rn(m_run[qq], mn));
           }
         }
         // P_hat^T: per query row q the 16-key block of this lane (lanes 0-15 / 16-31); even
