@@ -183,9 +183,8 @@ struct StreamCfg {
   static constexpr int NS = 3;                        // stages
   static constexpr uint32_t OFF_RTAB = NS * STAGE;
   static constexpr uint32_t OFF_BAR = OFF_RTAB + 1024;
-  static constexpr uint32_t OFF_POS = OFF_BAR + 16 * NS + 16;     // [NS] int4 chunk positions
   static constexpr int SC_MAX = 2048;                             // Smooth-QK floats per tensor kept in smem
-  static constexpr uint32_t OFF_SC = OFF_POS + 16 * NS;           // [2][SC_MAX] fp32: s, then s_inv
+  static constexpr uint32_t OFF_SC = OFF_BAR + 16 * NS + 16;      // [2][SC_MAX] fp32: s, then s_inv
   static constexpr uint32_t SMEM = OFF_SC + 2 * SC_MAX * 4 + 128; // + slack for 128-B alignment
 };
 
@@ -282,9 +281,9 @@ __device__ __forceinline__ void unpack16(const uint8_t* src, float2 (&v)[8]) {
   for (int e = 0; e < 8; ++e) v[e] = __bfloat1622float2(p2[e]);
 }
 
-// Per-thread loads of a row chunk that do not depend on its data (issued before the wait
-// for the chunk's bytes): the Smooth-QK scales of the thread's channels and, with ROPE,
-// the angle-table columns of its channel pairs.
+// Per-thread loads of a row chunk that do not depend on its data, issued before the wait
+// for the chunk's bytes (every warp splits the chunk index itself): the Smooth-QK scales
+// of the thread's channels and, with ROPE, the angle-table columns of its channel pairs.
 template <int D, bool ROPE>
 struct RowPrefetch {
   float4 sc4[ROPE ? 8 : 4];                           // [0..3] block 1 (ROPE: first half), [4..7] ROPE second half
@@ -433,7 +432,6 @@ __global__ void __launch_bounds__(256, ROPE ? 2 : 3) k_quant_stream(QuantRowsArg
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* empty = full + C::NS;
   volatile int* abort = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 16 * C::NS);
-  int4* pos = reinterpret_cast<int4*>(smem + C::OFF_POS);   // [NS] chunk positions
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   fill_recip_table(rtab, threadIdx.x, 256);
   // the Smooth-QK scales of Q and K in shared memory when they fit (Hkv * D <= SC_MAX)
@@ -461,12 +459,8 @@ __global__ void __launch_bounds__(256, ROPE ? 2 : 3) k_quant_stream(QuantRowsArg
   const int total = qa.units + ka.units + va.units, G = gridDim.x, b0 = blockIdx.x;
   const int mine = b0 < total ? (total - 1 - b0) / G + 1 : 0;   // chunks of this CTA
   int issued = 0;
-  // warp 0 splits each chunk index once, when it issues the copy, and leaves the position
-  // in the stage's slot for the other warps (ordered by the stage's full barrier)
   auto issue = [&](int j, int st) {
-    const ChunkPos cp = chunk_pos<D>(b0 + j * G, qa, ka, dv);
-    if (lane == 0) pos[st] = make_int4(cp.kind, cp.bh, cp.h, cp.r0);
-    stream_issue<D>(cp, qa, ka, va, smem + st * C::STAGE, &full[st]);
+    stream_issue<D>(chunk_pos<D>(b0 + j * G, qa, ka, dv), qa, ka, va, smem + st * C::STAGE, &full[st]);
   };
   if (warp == 0) {
     for (; issued < C::NS && issued < mine; ++issued) issue(issued, issued);
@@ -476,19 +470,19 @@ __global__ void __launch_bounds__(256, ROPE ? 2 : 3) k_quant_stream(QuantRowsArg
   for (int i = 0; i < mine; ++i) {
     const int st = i % C::NS;
     const uint32_t par = (i / C::NS) & 1;
+    // the chunk's position and the loads that do not depend on its bytes come before
+    // the wait for them
+    const ChunkPos p = chunk_pos<D>(b0 + i * G, qa, ka, dv);
+    const QuantRowsArgs& a = p.kind == 0 ? qa : ka;
+    const int g = p.kind == 2 ? 0 : (int)fdiv((uint32_t)p.h, p.kind == 0 ? dv.q_group : dv.k_group);
+    RowPrefetch<D, ROPE> f;
+    if (p.kind != 2) stream_prefetch<D, ROPE>(a, p.kind == 0 ? scale_q : scale_k, p, g, f);
     ok = __all_sync(0xffffffffu, mbar_wait(&full[st], par, abort, status, wait_ns));
     if (!ok) break;
-    const int4 pv = pos[st];
-    ChunkPos p;
-    p.kind = pv.x, p.bh = pv.y, p.h = pv.z, p.r0 = pv.w, p.b = 0;
     const uint8_t* stage = smem + st * C::STAGE;
     if (p.kind == 2) {
       stream_vt<D>(va, p, stage, rtab, nan_acc);
     } else {
-      const QuantRowsArgs& a = p.kind == 0 ? qa : ka;
-      const int g = (int)fdiv((uint32_t)p.h, p.kind == 0 ? dv.q_group : dv.k_group);
-      RowPrefetch<D, ROPE> f;
-      stream_prefetch<D, ROPE>(a, p.kind == 0 ? scale_q : scale_k, p, g, f);
       stream_rows<D, ROPE>(a, p, f, stage, rtab, nan_acc);
     }
     __syncwarp();
