@@ -19,7 +19,7 @@ def test_device_codec_and_exp2_match_oracle():
     rng = np.random.default_rng(11)
     ex = np.concatenate([rng.uniform(-130, 1, 3_000_000).astype(np.float32),
                          np.arange(0xBF800000, 0xC0000000, 37, dtype=np.uint32).view(np.float32),
-                         np.array([-np.inf, -127.0, -126.0, 0.0, -0.0], np.float32)])
+                         np.array([-np.inf, -127.0, -126.0, 0.0, -0.0, np.nan], np.float32)])
     allx = np.concatenate([x, ex]).astype(np.float32)
     e2, e4, e = th.probe_codec(gc.to_dev(allx))
     e2, e4, e = e2.cpu().numpy(), e4.cpu().numpy(), e.cpu().numpy()
