@@ -558,6 +558,17 @@ def run_gpu(args):
     fp4_nominal = bf16 * FP4_OVER_BF16
     fp4_peak = fp4["burst_tflops"]
     achieved = flops / (k_attn * 1e-3) / 1e12
+    # the resource that actually binds the attention kernel: the softmax's FP32 work.  The
+    # plain P_hat rounding costs 8 FP32 lane operations per visible score (the fma of
+    # S c - m, the round-down add, the subtraction and the fma of the range split, the three
+    # fmas of the cubic, the product with RN(1/sigma)); the FP32 pipes of the GPU run
+    # SMs x 128 lanes per cycle at the sampled SM clock
+    vis = sum((b1 - b0) * (g1 - g0) * G * (N * (N + 1) // 2 if w.causal else N * N) for b0, b1, g0, g1 in blocks)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    sm_hz = (clk.get("sm_mhz") or 1965.0) * 1e6
+    fp32_lane_ops = 8.0 * vis
+    fp32_achieved = fp32_lane_ops / (k_attn * 1e-3) / 1e12
+    fp32_peak = sms * 128 * sm_hz / 1e12
     # algorithmic HBM bytes of one attention launch: 4-bit Q, K, V^T (codes + scales) read,
     # bf16 O and fp16 m, l written
     # (summed over the rank's blocks of heads)
@@ -607,6 +618,12 @@ def run_gpu(args):
                              "algorithmic_bytes": rope_bytes,
                              "note": "pre-RoPE bf16 Q, K read, 4-bit codes + scales written (2.5625 B/elem); "
                                      "the fp32 angle tables stay in L2"},
+        "softmax_fp32": {"achieved": round(fp32_achieved, 2), "peak": round(fp32_peak, 2),
+                         "unit": "T lane-ops/s", "frac": round(fp32_achieved / fp32_peak, 4),
+                         "lane_ops_per_launch": fp32_lane_ops,
+                         "note": "attention kernel: 8 FP32 lane operations of the plain P_hat rounding per "
+                                 "visible score / its event time, against SMs x 128 FP32 lanes x the sampled "
+                                 "SM clock; the integer exponent insert and the clamp are not counted"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                      "traffic": ATTN_TRAFFIC_BYTES if whole_call else None,
