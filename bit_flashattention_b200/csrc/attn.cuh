@@ -77,13 +77,11 @@ struct AttnCfg {
   static_assert(T_END <= 512, "TMEM budget exceeded");
   static_assert(D == 64 || D == 128 || D == 256, "head dim");
   static_assert(BC == 64 || BC == 128 || BC == 256, "kv tile");
-  // softmax warpgroups: each takes CW consecutive score columns of every row and D/NSW
-  // columns of O (both at least 32, the width of one tcgen05.ld)
-#ifndef HIFA4_MAX_NSW
-#define HIFA4_MAX_NSW 4
-#endif
+  // softmax warpgroups (at most 4, so that all softmax warps of a lane quarter share one
+  // SMSP): each takes CW consecutive score columns of every row and D/NSW columns of O (both
+  // at least 32, the width of one tcgen05.ld)
   static constexpr int NSW0 = (BC < D ? BC : D) / 32;
-  static constexpr int NSW = NSW0 < HIFA4_MAX_NSW ? NSW0 : HIFA4_MAX_NSW, CW = BC / NSW;
+  static constexpr int NSW = NSW0 < 4 ? NSW0 : 4, CW = BC / NSW;
   static_assert(NSW == 2 || NSW == 4, "softmax warpgroups");
   static_assert(CW == 32 || CW == 64 || CW == 128, "column split");
   static constexpr int NTHREADS = 96 + 128 * NSW;   // producer, QK^T issuer, PV issuer, softmax
